@@ -1,0 +1,442 @@
+"""RecSA build -> select -> attend benchmark on B200 (one JSON line on rank 0).
+
+Default workload: 524288-token decode, 4 independent sequences, one appended token
+per sequence per step (recsa_append then recsa_decode), Qwen3-4B attention shapes
+(32 query heads, 8 KV heads, d = 128), C = 16, k = 256, bf16 storage.  Metric:
+decode tokens/s (all sequences, all GPUs).  The 4096-query prefill chunk at 524K
+is measured in the same run and reported under "prefill".
+
+Multi-GPU: every rank runs its own 4 sequences (weak scaling, no collective in
+the data path); the time is the max over ranks.
+
+--impl reference runs the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only) and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
+HBM_NOMINAL_GBS = 8000.0
+
+# workload: 524K decode, B = 4 (and the 4096-query prefill chunk at 524K)
+W = dict(Hq=32, Hkv=8, d=128, C=16, k=256, L=524288, B=4, dtype="bf16", base=1e6,
+         prefill_q=4096)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def step_bytes(counts, k, s_vec, B, Hkv, Hq, d, esize):
+    """Algorithmic bytes of one decode step from the per-(b, kvh) list sizes:
+    keys scored ((|A|-1) rows) and summary values (|A|-k rows) of every scored
+    level, level-0 K and V rows, plus q, out and the appended rows."""
+    tot = 0
+    per_level = {}
+    for b in range(counts.shape[0]):
+        for h in range(counts.shape[1]):
+            c = counts[b, h]
+            for l in range(1, len(c)):
+                if c[l] > 0:
+                    by = ((c[l] - 1) + (c[l] - min(k, c[l]))) * s_vec
+                    per_level[l] = per_level.get(l, 0) + by
+                    tot += by
+            per_level[0] = per_level.get(0, 0) + 2 * c[0] * s_vec
+            tot += 2 * c[0] * s_vec
+    io = B * Hq * d * esize * 2 + B * Hkv * 2 * d * esize
+    return tot + io, per_level
+
+
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    import torch
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    import torch
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def run_ours(args):
+    import torch
+    from long_context_recsa_b200 import build, inputs as I
+    build.build()
+    import long_context_recsa_b200.recsa as R
+
+    ws, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, Hq, Hkv, d, C, k, L = W["B"], W["Hq"], W["Hkv"], W["d"], W["C"], W["k"], W["L"]
+    S = args.warmup + args.steps
+    cap = L + S + 16
+    dt = I.torch_dtype(W["dtype"])
+    esize = 2
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype=W["dtype"],
+                   rope_base=W["base"], pooler_w=I.pooler_w(C).tolist())
+    # inputs resident in HBM before timing (seeded, per rank)
+    g = torch.Generator(device=dev)
+    g.manual_seed(I.slice_seed(3, I.STREAM_K, 0, 0) + 7919 * rank)
+    K = torch.randn(B, Hkv, cap, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    V = torch.randn(B, Hkv, cap, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    knew = torch.randn(S, B, Hkv, 1, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    vnew = torch.randn(S, B, Hkv, 1, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    qs = torch.randn(S, B, Hq, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    tree = R.RecsaTree(cfg, cap, B, max_queries=max(B, 64), k0=K, v0=V)
+
+    # tree build from raw K, V (reported separately)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    tree.recsa_build([L] * B)
+    e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    build_bytes = B * Hkv * L * d * esize * 2 * (1 + 1 / 15.0)
+
+    # one decode step = append + decode, captured once; device-side lengths make
+    # the graph replayable step after step
+    kst = torch.empty(B, Hkv, 1, d, dtype=dt, device=dev)
+    vst = torch.empty_like(kst)
+    qst = torch.empty(B, Hq, d, dtype=dt, device=dev)
+    out = torch.empty_like(qst)
+    cnt = torch.zeros(B, Hkv, tree.n_sel_levels + 1, dtype=torch.int32, device=dev)
+    prof_ev = {}
+    for which in [0] + list(range(1, tree.n_sel_levels + 1)) + [-1, -2]:
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); b_.record()
+        prof_ev[which] = (a, b_)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    graphs = {}
+    for which, (a, b_) in prof_ev.items():
+        tree.recsa_set_profile_events(which, a, b_)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gr, stream=stream):
+                tree.recsa_append(kst, vst)
+                tree.recsa_decode(qst, out, None, cnt)
+        graphs[which] = gr
+    tree.recsa_set_profile_events(0, None, None)
+    torch.cuda.synchronize()
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    launches_per_step = 1 + tree.n_sel_levels + 2
+    step_ms, kern_ms = [], {w: [] for w in prof_ev}
+    whiches = list(prof_ev)
+
+    def one_step(i, timed):
+        which = whiches[i % len(whiches)]
+        kst.copy_(knew[i]); vst.copy_(vnew[i]); qst.copy_(qs[i])
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        graphs[which].replay()
+        s1.record()
+        s1.synchronize()
+        if timed:
+            step_ms.append(s0.elapsed_time(s1))
+            a, b_ = prof_ev[which]
+            kern_ms[which].append(a.elapsed_time(b_))
+
+    for i in range(args.warmup):
+        one_step(i, False)
+    barrier(ws)
+    with ClockSampler(local) as clk:
+        for i in range(args.warmup, S):
+            one_step(i, True)
+        barrier(ws)
+    assert tree.recsa_get_status() == R.RECSA_OK
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
+    value = ws * B / (ms / 1e3)
+    counts = cnt.cpu().numpy()
+    by_step, per_level = step_bytes(counts, k, d * esize, B, Hkv, Hq, d, esize)
+    hbm, peak_kind = peaks()
+    kern_avg = {w: (sum(v) / len(v) if v else None) for w, v in kern_ms.items()}
+    # dominant kernel: the one with the largest share of the step
+    dom = max((w for w in kern_avg if w >= 0 and kern_avg[w]), key=lambda w: kern_avg[w])
+    dom_bytes = per_level.get(dom, 0)
+    achieved = dom_bytes / (kern_avg[dom] / 1e3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: K,V,q,new k/v ~ N(0,1) seeded, resident in HBM",
+        "config": {"workload": "decode 524K ctx, batch 4, append 1 token/seq/step, "
+                               "Hq=32 Hkv=8 d=128 C=16 k=256 bf16",
+                   "seq_len": L, "global_batch": B * ws, "parallelism": f"replicas x{ws}",
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "timing": "per-step CUDA events around one graph replay"},
+        "bytes_per_step": int(by_step),
+        "hbm_frac_of_nominal_8TBs": round(by_step / (ms / 1e3) / 1e9 / HBM_NOMINAL_GBS, 4),
+        "hbm_frac_of_measured": round(by_step / (ms / 1e3) / 1e9 / hbm, 4),
+        "roofline": {"bound": "hbm", "kernel": f"level{dom}_kernel",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": None,
+                     "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": int(dom_bytes),
+                     "avg_launch_ms": round(kern_avg[dom], 5)},
+        "kernel_ms": {("append" if w == -1 else "combine" if w == -2 else f"level{w}"):
+                      (round(v, 5) if v else None) for w, v in kern_avg.items()},
+        "build_524k": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_e2e:
+        res["e2e"] = e2e_decode(tree, R, knew, vnew, qs, args, ws, flush)
+    if not args.no_prefill:
+        res["prefill"] = bench_prefill(R, I, cfg, K, V, tree, args, ws, dev, flush)
+    if rank == 0:
+        res["cpu_baseline"] = cpu_baseline(K, V, qs, cfg, R)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        del graphs
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def e2e_decode(tree, R, knew, vnew, qs, args, ws, flush):
+    """Public-API path with host buffers: per step pinned H2D of the new k, v and q,
+    recsa_append + recsa_decode, D2H of the output; timed with events."""
+    import torch
+    S = knew.shape[0]
+    n = min(args.steps, 20)
+    hk = knew[:n].cpu().pin_memory()
+    hv = vnew[:n].cpu().pin_memory()
+    hq = qs[:n].cpu().pin_memory()
+    dk = torch.empty_like(knew[0]); dv = torch.empty_like(vnew[0]); dq = torch.empty_like(qs[0])
+    dout = torch.empty_like(dq)
+    hout = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+    # rewind the tree to the benchmark length by rebuilding (outside timing)
+    tree.recsa_build([W["L"]] * W["B"])
+    torch.cuda.synchronize()
+    times = []
+    for i in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dk.copy_(hk[i], non_blocking=True); dv.copy_(hv[i], non_blocking=True)
+        dq.copy_(hq[i], non_blocking=True)
+        tree.recsa_append(dk, dv)
+        tree.recsa_decode(dq, dout)
+        hout.copy_(dout, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = max_over_ranks(sum(times) / len(times), ws)
+    es = dq.element_size()
+    return {"value": round(ws * W["B"] / (ms / 1e3), 1), "unit": "tok/s", "ms_per_step": round(ms, 5),
+            "h2d_bytes_per_step": int((dk.numel() + dv.numel() + dq.numel()) * es),
+            "d2h_bytes_per_step": int(dout.numel() * es), "steps": n}
+
+
+def bench_prefill(R, I, cfg, K, V, tree_decode, args, ws, dev, flush):
+    """4096 causal queries at positions 520192..524287 of the 524288-token tree."""
+    import torch
+    nq = W["prefill_q"]
+    L = W["L"]
+    # a batch-1 view of the first sequence for the chunk
+    pt = R.RecsaTree(cfg, K.shape[2], 1, max_queries=1024, k0=K[:1], v0=V[:1])
+    pt.recsa_build([L])
+    g = torch.Generator(device=dev)
+    g.manual_seed(I.slice_seed(4, I.STREAM_Q, 0, 0))
+    Q = torch.randn(1, nq, W["Hq"], W["d"], generator=g, device=dev).to(cfg.torch_dtype)
+    O = torch.empty_like(Q)
+    for _ in range(2):
+        pt.recsa_prefill_chunk(Q, L - nq, O)
+    torch.cuda.synchronize()
+    reps = 3
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pt.recsa_prefill_chunk(Q, L - nq, O)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    assert pt.recsa_get_status() == R.RECSA_OK
+    ms = max_over_ranks(sum(times) / len(times), ws)
+    return {"value": round(ws * nq / (ms / 1e3), 1), "unit": "tok/s", "ms_per_chunk": round(ms, 3),
+            "workload": "4096-query chunk at positions 520192..524287 of a 524288-token tree, "
+                        "batch 1, same shapes", "path": "per-query select/attend kernels"}
+
+
+def cpu_baseline(K, V, qs, cfg, R):
+    """The fp64 oracle on a bounded sample: select + attend of decode queries of one
+    (sequence, KV head) unit over its pre-built fp64 tree (tree build excluded)."""
+    import numpy as np
+    import torch
+    from oracle import recsa_oracle as O
+    cores = len(os.sched_getaffinity(0))
+    L, C, k, G, d = W["L"], W["C"], W["k"], W["Hq"] // W["Hkv"], W["d"]
+    Kh = K[0, 0, :L].double().cpu().numpy()
+    Vh = V[0, 0, :L].double().cpu().numpy()
+    levels = O.build_tree(Kh, Vh, C, np.asarray(cfg.pooler_w, dtype=np.float64), "bf16")
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        q = qs[n % qs.shape[0], 0, :G].double().cpu().numpy()
+        O.select_and_attend(levels, q, L - 1, C, k, base=W["base"])
+        n += 1
+        el = time.perf_counter() - t0
+        if el > 10.0 or n >= 200:
+            break
+    per_unit = el / n
+    units_per_token = W["Hkv"]
+    return {"value": round(1.0 / (per_unit * units_per_token), 3), "unit": "tok/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} decode queries (select+attend, fp64) of one (sequence, KV head) unit "
+                      f"at t=524287 over a pre-built tree; scaled by 8 units per token; "
+                      f"tree build/append excluded"}
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    from long_context_recsa_b200 import inputs as I
+    from oracle import recsa_oracle as O
+    cores = len(os.sched_getaffinity(0))
+    L, C, k, Hq, Hkv, d = W["L"], W["C"], W["k"], W["Hq"], W["Hkv"], W["d"]
+    G = Hq // Hkv
+    Ks, Vs = I.kv_slice(3, 0, 0, L, d, "bf16")
+    levels = O.build_tree(Ks.double().numpy(), Vs.double().numpy(), C,
+                          I.pooler_w(C).double().numpy(), "bf16")
+    q = I.q_rows(3, 0, args.warmup + args.steps, Hq, d, "bf16").double().numpy()
+    for i in range(args.warmup):
+        O.select_and_attend(levels, q[i, :G], L - 1, C, k, base=W["base"])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        O.select_and_attend(levels, q[args.warmup + i, :G], L - 1, C, k, base=W["base"])
+    el = (time.perf_counter() - t0) / args.steps
+    tok_s = 1.0 / (el * Hkv)
+    res = {"impl": "reference", "metric": METRIC, "value": round(tok_s, 3), "unit": "tok/s",
+           "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(el * Hkv * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": "decode 524K ctx, Hq=32 Hkv=8 d=128 C=16 k=256 (oracle sample)",
+                      "seq_len": L},
+           "cpu_baseline": {"value": round(tok_s, 3), "unit": "tok/s", "cores": cores,
+                            "kind": "oracle",
+                            "sample": "per step: select+attend of one decode query for one "
+                                      "(sequence, KV head) unit, scaled by 8 units per token; "
+                                      "tree built once before timing"},
+           "e2e": {"value": round(tok_s, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

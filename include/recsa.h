@@ -1,0 +1,205 @@
+/*
+ * recsa.h -- C ABI of the RecSA (Recursive Sparse Attention) build -> select ->
+ * attend hot path, hand-written CUDA for sm_100a (B200).  Library: librecsa.so.
+ *
+ * Method: "Recursive Sparse Attention: Million-Token Length Extrapolation at
+ * Logarithmic Cost" (arXiv:2611.07232).  Tree construction is Eq.1 ("Tree
+ * Construction"), top-down selection Eq.3 ("Hierarchical Selection") with
+ * candidate-local RoPE ("Key Theoretical Insight"), and the unified softmax over
+ * level-0 tokens and unselected summaries Eq.4 ("Unified Softmax").
+ *
+ * Conventions for every call:
+ *   - Device buffers are allocated and owned by the caller.  The library owns only
+ *     the small host handle returned by recsa_tree_init.  It never calls cudaMalloc.
+ *   - Calls that take a stream are asynchronous on that stream (a cudaStream_t,
+ *     passed as void*; NULL is the legacy default stream) and issue only kernel
+ *     launches, so they can be captured in a CUDA graph.  recsa_get_status is the
+ *     one call that synchronises.
+ *   - Argument, shape, alignment and capacity errors are detected on the host and
+ *     returned before anything is launched.  Conditions only the device can see (a
+ *     query position beyond the current length after graph replays, a length that
+ *     would pass the capacity) set a sticky device status word and the affected
+ *     work is skipped; recsa_get_status reports it.  Kernels never trap.
+ *   - Layouts are row-major with the head dimension d contiguous.  Element type of
+ *     K, V, q, out and the level tables is the config's dtype (fp32 or bf16).
+ */
+#ifndef RECSA_H
+#define RECSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RECSA_API __attribute__((visibility("default")))
+#else
+#define RECSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RECSA_OK = 0,
+    RECSA_E_INVAL = 1,        /* NULL pointer, bad size, misaligned pointer/stride, bad config   */
+    RECSA_E_UNSUPPORTED = 2,  /* valid but not built here: head_dim, group size, C, k, C*k       */
+    RECSA_E_CAPACITY = 3,     /* a length would exceed capacity, or a buffer is too small        */
+    RECSA_E_CUDA = 4,         /* a CUDA runtime call or kernel launch failed                      */
+    RECSA_E_TIMEOUT = 5,      /* a bounded device wait gave up                                    */
+    RECSA_E_DEVICE = 6        /* device status word: a query or append was out of range          */
+} recsa_status;
+
+typedef enum { RECSA_F32 = 0, RECSA_BF16 = 1 } recsa_dtype;
+
+#define RECSA_MAX_C 32
+#define RECSA_MAX_BATCH 64
+#define RECSA_MAX_LEVELS 32
+
+/* Method and shape parameters.
+ *   head_dim   d, 64 or 128.
+ *   n_q_heads  Hq; n_kv_heads Hkv; Hq/Hkv = G in {1, 2, 4, 8}.  Query head h reads
+ *              KV head h / G (contiguous groups); the G heads of a group share one
+ *              selection, scored by the mean of their logits (GQA stand-in, since
+ *              the importance I of Eq.3 is not defined on the pages).
+ *   C          branching factor of the tree, 2..32 (the pages use 16).
+ *   k          per-level selection budget, 1..512 (the pages use 256); C*k <= 8192.
+ *   dtype      storage of K, V, q, outputs and level tables (recsa_dtype).
+ *   rope_base  RoPE base b > 1: pair (j, j+d/2) turns by pos * b^(-2j/d).
+ *   scale      logit scale; 0 selects 1/sqrt(d).
+ *   pooler_w   pooler logits w[0..C-1].  Stand-in pooler: a parent key is
+ *              sum_c softmax(w)_c K_child_c over its present children (Eq.1 with
+ *              Pool fixed to a softmax-weighted sum shared by all levels/heads). */
+typedef struct {
+    int32_t head_dim;
+    int32_t n_q_heads;
+    int32_t n_kv_heads;
+    int32_t C;
+    int32_t k;
+    int32_t dtype;
+    double rope_base;
+    float scale;
+    float pooler_w[RECSA_MAX_C];
+} recsa_config;
+
+typedef struct recsa_tree recsa_tree;   /* opaque host handle; does not own device memory */
+
+/* Sizes of the caller-allocated buffers for a tree of `capacity` tokens per
+ * sequence, `batch` sequences and at most `max_queries` queries per kernel wave
+ * (decode uses `batch` queries; prefill chunks are processed in waves of
+ * max_queries).  Pure host computation.
+ *   level_bytes      bytes for the level tables (levels 1.. up to a single root).
+ *   workspace_bytes  bytes for the workspace (status word, device lengths, RoPE
+ *                    table, per-level selections, split-softmax partials).
+ *   n_levels         number of tree levels at capacity, level 0 included.
+ * Any output pointer may be NULL.  Errors: RECSA_E_INVAL, RECSA_E_UNSUPPORTED. */
+RECSA_API recsa_status recsa_query_sizes(const recsa_config* cfg, int64_t capacity, int32_t batch,
+                               int32_t max_queries, size_t* level_bytes,
+                               size_t* workspace_bytes, int32_t* n_levels);
+
+/* Bind a tree to caller memory and initialise its workspace on `stream` (status
+ * word cleared, all lengths 0, RoPE cos/sin table for positions [0, C*k) computed
+ * in fp64 and stored fp32).
+ *   k0, v0      level-0 KV cache, element (b, h, t, :) at base + b*s[0] + h*s[1]
+ *               + t*s[2] elements, d contiguous.  16-byte aligned; each stride a
+ *               multiple of 16 bytes; s[2] >= d.  The library writes rows here
+ *               only in recsa_append.
+ *   kv_strides  s[3] in elements (host array, copied).
+ *   levels      level tables, >= level_bytes, 256-byte aligned.  Level l >= 1 of
+ *               KV head h of sequence b is a [rows_l][d] K table and a [rows_l][d]
+ *               V table (recsa_level_info gives offsets).
+ *   workspace   >= workspace_bytes, 256-byte aligned.
+ * On success *out receives a new handle (free with recsa_tree_free). */
+RECSA_API recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t batch,
+                             int32_t max_queries, void* k0, void* v0,
+                             const int64_t kv_strides[3], void* levels, size_t level_bytes,
+                             void* workspace, size_t workspace_bytes, void* stream,
+                             recsa_tree** out);
+
+/* Eq.1 over the whole cache: set the length of sequence b to lengths[b] (host
+ * array of `batch` values, 0 <= lengths[b] <= capacity) and compute every level
+ * l >= 1 from level 0.  Node i of level l pools children C*i .. min(C*i+C-1,
+ * n_{l-1}-1): K = sum_c alpha_c K_c with alpha = softmax(w) over the m present
+ * children, V = (1/m) sum_c V_c, accumulated in fp64 and rounded once (to nearest
+ * even) to the storage dtype; the next level pools the rounded values. */
+RECSA_API recsa_status recsa_build(recsa_tree* tree, const int64_t* lengths, void* stream);
+
+/* Append n >= 1 tokens to every sequence: k_new, v_new are device arrays
+ * [batch][Hkv][n][d] (contiguous, 16-byte aligned).  Rows are written at the
+ * device-side length L of each sequence, then every ancestor node of the new
+ * tokens is re-pooled exactly as recsa_build would compute it (build(L) followed
+ * by append(n) is bitwise equal to build(L+n)), and L grows by n.  If L + n would
+ * exceed capacity the sequence is left unchanged and the status word records
+ * RECSA_E_CAPACITY (the host also rejects this synchronously while its own copy
+ * of the lengths is current, i.e. outside graph replays). */
+RECSA_API recsa_status recsa_append(recsa_tree* tree, const void* k_new, const void* v_new, int32_t n,
+                          void* stream);
+
+/* Decode one query per sequence at its last position t = L_b - 1 (so the newest
+ * token attends to itself).
+ *   q        [batch][Hq][d] device, 16-byte aligned.
+ *   out      [batch][Hq][d] device: Eq.4 output, rounded to the storage dtype.
+ *            A sequence of length 0 gets zeros.
+ *   sel_out  optional [batch][Hkv][NL][k] int32: selected node indices S^(l) of
+ *            scored level l at index l-1 (ascending, current node last, -1 where
+ *            unused or where the level is above the first scored level).  NL is
+ *            recsa_tree_info's n_sel_levels.
+ *   counts_out optional [batch][Hkv][NL+1] int32: |A^(l)| at index l for levels
+ *            that are scored (index 0: the level-0 list), 0 above them. */
+RECSA_API recsa_status recsa_decode(recsa_tree* tree, const void* q, void* out, int32_t* sel_out,
+                          int32_t* counts_out, void* stream);
+
+/* Causal queries of a chunk: row i of sequence b sits at position pos0 + i and
+ * must already be in the tree (pos0 + n <= L_b).
+ *   Q  [batch][n][Hq][d] device;  O [batch][n][Hq][d] device.
+ *   sel_out / counts_out as in recsa_decode with batch*n queries (b-major).
+ * Each row equals recsa_decode of a tree holding only tokens [0..pos0+i]. */
+RECSA_API recsa_status recsa_prefill_chunk(recsa_tree* tree, const void* Q, int64_t pos0, int32_t n,
+                                 void* O, int32_t* sel_out, int32_t* counts_out, void* stream);
+
+/* Synchronise `stream`, read and clear the device status word.  Returns RECSA_OK or
+ * the first device-side error recorded since the last call. */
+RECSA_API recsa_status recsa_get_status(recsa_tree* tree, void* stream);
+
+typedef struct {
+    int32_t n_levels;       /* levels stored at capacity, level 0 included           */
+    int32_t n_sel_levels;   /* NL: highest level that any position can score         */
+    int32_t splits;         /* CTAs (a thread-block cluster) per unit for levels >= 1 */
+    int32_t splits0;        /* CTAs per unit for level 0                               */
+    int64_t capacity;
+    int32_t batch;
+    int32_t max_queries;
+} recsa_tree_info_t;
+
+RECSA_API recsa_status recsa_tree_info(const recsa_tree* tree, recsa_tree_info_t* info);
+
+/* Where level `level` (1 <= level < n_levels) lives inside the `levels` buffer:
+ * byte offsets of its K and V tables and rows per (sequence, KV head).  Row i of
+ * head h of sequence b is at offset + ((b*Hkv + h)*rows + i)*d*elem_size. */
+RECSA_API recsa_status recsa_level_info(const recsa_tree* tree, int32_t level, int64_t* k_offset,
+                              int64_t* v_offset, int64_t* rows);
+
+/* Host lengths as the library last set them (exact unless a captured graph was
+ * replayed since).  lengths: host array of batch values. */
+RECSA_API recsa_status recsa_host_lengths(const recsa_tree* tree, int64_t* lengths);
+
+/* Kernel timing hook.  From the next call on, record CUDA event `start` (a
+ * cudaEvent_t, created by the caller with timing enabled) on the call's stream just
+ * before the kernel selected by `which` is launched and `stop` just after it:
+ *   which = l in [0, n_sel_levels]: the select/attend kernel of level l (0 = the
+ *           level-0 attention), in recsa_decode and in each prefill wave;
+ *   which = -1: the append kernel(s) of recsa_append;  -2: the combine kernel.
+ * Records use cudaEventRecordExternal, so they also become event nodes when the
+ * call is captured in a CUDA graph.  start = stop = NULL clears the hook.
+ * No device memory is touched. */
+RECSA_API recsa_status recsa_set_profile_events(recsa_tree* tree, int32_t which, void* start,
+                                                void* stop);
+
+/* Free the host handle.  Device memory stays with the caller. */
+RECSA_API recsa_status recsa_tree_free(recsa_tree* tree);
+
+RECSA_API const char* recsa_status_str(recsa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RECSA_H */

@@ -1,0 +1,338 @@
+// Host side of the RecSA C ABI: argument checks, buffer layout, kernel dispatch.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "recsa_internal.cuh"
+
+namespace recsa {
+
+constexpr int kSplits = 8;    // CTAs (one thread-block cluster) per unit, levels >= 1
+constexpr int kSplits0 = 8;   // CTAs per unit at level 0
+
+struct Layout {
+    int esize, D, G;
+    int n_levels;
+    int64_t rows[kMaxLevels];
+    int64_t off_k[kMaxLevels], off_v[kMaxLevels];
+    size_t level_bytes;
+    int NL, SPL, NS0, NSLOT;
+    size_t o_status, o_lens, o_done, o_rope, o_sel, o_cnt, o_part, ws_bytes;
+};
+
+static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static recsa_status check_config(const recsa_config* c) {
+    if (!c) return RECSA_E_INVAL;
+    if (c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->n_q_heads % c->n_kv_heads) return RECSA_E_INVAL;
+    if (c->C < 2 || c->k < 1) return RECSA_E_INVAL;
+    if (c->dtype != RECSA_F32 && c->dtype != RECSA_BF16) return RECSA_E_INVAL;
+    if (!(c->rope_base > 1.0) || !isfinite(c->rope_base)) return RECSA_E_INVAL;
+    if (!(c->scale >= 0.0f) || !isfinite(c->scale)) return RECSA_E_INVAL;
+    if (c->head_dim != 64 && c->head_dim != 128) return RECSA_E_UNSUPPORTED;
+    const int G = c->n_q_heads / c->n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return RECSA_E_UNSUPPORTED;
+    if (c->C > RECSA_MAX_C || c->k > 512 || (int64_t)c->C * c->k > 8192) return RECSA_E_UNSUPPORTED;
+    for (int i = 0; i < c->C; ++i)
+        if (!isfinite(c->pooler_w[i])) return RECSA_E_INVAL;
+    return RECSA_OK;
+}
+
+static recsa_status compute_layout(const recsa_config* c, int64_t cap, int B, int Qmax, Layout* L) {
+    recsa_status st = check_config(c);
+    if (st != RECSA_OK) return st;
+    if (cap < 1 || cap > ((int64_t)1 << 40)) return RECSA_E_INVAL;
+    if (B < 1 || B > RECSA_MAX_BATCH) return RECSA_E_INVAL;
+    if (Qmax < B || Qmax > (1 << 20)) return RECSA_E_INVAL;
+    memset(L, 0, sizeof(*L));
+    L->esize = c->dtype == RECSA_BF16 ? 2 : 4;
+    L->D = c->head_dim;
+    L->G = c->n_q_heads / c->n_kv_heads;
+    const int Hkv = c->n_kv_heads;
+    L->rows[0] = cap;
+    int n = 1;
+    while (L->rows[n - 1] > 1) {
+        if (n >= kMaxLevels - 2) return RECSA_E_UNSUPPORTED;
+        L->rows[n] = (L->rows[n - 1] + c->C - 1) / c->C;
+        ++n;
+    }
+    L->n_levels = n;
+    size_t o = 0;
+    for (int l = 1; l < n; ++l) {
+        const size_t bytes = al256((size_t)B * Hkv * L->rows[l] * L->D * L->esize);
+        L->off_k[l] = (int64_t)o;
+        o += bytes;
+        L->off_v[l] = (int64_t)o;
+        o += bytes;
+    }
+    L->level_bytes = o > 0 ? o : 256;
+    // highest level any position t < cap can score: floor(t / C^l) >= k
+    int NL = 0;
+    {
+        int64_t p = cap - 1;
+        int l = 0;
+        while (p > 0) {
+            p /= c->C;
+            ++l;
+            if (p >= c->k) NL = l;
+        }
+    }
+    L->NL = NL;
+    L->SPL = kSplits;
+    L->NS0 = kSplits0;
+    L->NSLOT = NL * L->SPL + L->NS0;
+    const int ck = c->C * c->k;
+    size_t w = 0;
+    L->o_status = w; w = al256(w + 64);
+    L->o_lens = w;   w = al256(w + sizeof(int64_t) * B);
+    L->o_done = w;   w = al256(w + sizeof(uint32_t) * B);
+    L->o_rope = w;   w = al256(w + sizeof(float2) * (size_t)ck * (L->D / 2));
+    L->o_sel = w;    w = al256(w + sizeof(int32_t) * (size_t)Qmax * Hkv * (NL > 0 ? NL : 1) * c->k);
+    L->o_cnt = w;    w = al256(w + sizeof(int32_t) * (size_t)Qmax * Hkv * (NL + 1));
+    L->o_part = w;   w = al256(w + sizeof(float) * (size_t)Qmax * Hkv * L->NSLOT * L->G * (L->D + 2));
+    L->ws_bytes = w;
+    return RECSA_OK;
+}
+
+}  // namespace recsa
+
+using namespace recsa;
+
+struct recsa_tree {
+    recsa_config cfg;
+    Layout L;
+    int64_t cap;
+    int B, Qmax;
+    TreeView tv;
+    WorkView wv;
+    int64_t host_len[RECSA_MAX_BATCH];
+    ProfHook prof;
+};
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static recsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RECSA_OK : RECSA_E_CUDA; }
+
+extern "C" {
+
+const char* recsa_status_str(recsa_status s) {
+    switch (s) {
+        case RECSA_OK: return "ok";
+        case RECSA_E_INVAL: return "invalid argument";
+        case RECSA_E_UNSUPPORTED: return "unsupported configuration";
+        case RECSA_E_CAPACITY: return "capacity exceeded or buffer too small";
+        case RECSA_E_CUDA: return "CUDA error";
+        case RECSA_E_TIMEOUT: return "device wait timed out";
+        case RECSA_E_DEVICE: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+recsa_status recsa_query_sizes(const recsa_config* cfg, int64_t capacity, int32_t batch,
+                               int32_t max_queries, size_t* level_bytes, size_t* workspace_bytes,
+                               int32_t* n_levels) {
+    Layout L;
+    recsa_status st = compute_layout(cfg, capacity, batch, max_queries, &L);
+    if (st != RECSA_OK) return st;
+    if (level_bytes) *level_bytes = L.level_bytes;
+    if (workspace_bytes) *workspace_bytes = L.ws_bytes;
+    if (n_levels) *n_levels = L.n_levels;
+    return RECSA_OK;
+}
+
+recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t batch,
+                             int32_t max_queries, void* k0, void* v0, const int64_t kv_strides[3],
+                             void* levels, size_t level_bytes, void* workspace,
+                             size_t workspace_bytes, void* stream, recsa_tree** out) {
+    if (!out) return RECSA_E_INVAL;
+    *out = nullptr;
+    Layout L;
+    recsa_status st = compute_layout(cfg, capacity, batch, max_queries, &L);
+    if (st != RECSA_OK) return st;
+    if (!k0 || !v0 || !kv_strides || !levels || !workspace) return RECSA_E_INVAL;
+    if (!aligned16(k0) || !aligned16(v0)) return RECSA_E_INVAL;
+    if (((uintptr_t)levels & 255u) || ((uintptr_t)workspace & 255u)) return RECSA_E_INVAL;
+    const int64_t sb = kv_strides[0], sh = kv_strides[1], stt = kv_strides[2];
+    const int64_t per16 = 16 / L.esize;
+    if (sb < 0 || sh < 0 || stt < L.D) return RECSA_E_INVAL;
+    if (sb % per16 || sh % per16 || stt % per16) return RECSA_E_INVAL;
+    if (level_bytes < L.level_bytes || workspace_bytes < L.ws_bytes) return RECSA_E_CAPACITY;
+
+    recsa_tree* t = (recsa_tree*)calloc(1, sizeof(recsa_tree));
+    if (!t) return RECSA_E_INVAL;
+    t->cfg = *cfg;
+    t->L = L;
+    t->cap = capacity;
+    t->B = batch;
+    t->Qmax = max_queries;
+    TreeView& tv = t->tv;
+    tv.k0 = k0; tv.v0 = v0; tv.k0w = k0; tv.v0w = v0;
+    tv.s_b = sb; tv.s_h = sh; tv.s_t = stt;
+    tv.levels = (char*)levels;
+    for (int l = 0; l < kMaxLevels; ++l) {
+        tv.off_k[l] = L.off_k[l];
+        tv.off_v[l] = L.off_v[l];
+        tv.rows[l] = L.rows[l];
+    }
+    tv.B = batch;
+    tv.Hkv = cfg->n_kv_heads;
+    tv.Hq = cfg->n_q_heads;
+    tv.G = L.G;
+    tv.D = L.D;
+    tv.C = cfg->C;
+    tv.k = cfg->k;
+    tv.n_levels = L.n_levels;
+    tv.cap = capacity;
+    tv.scale = cfg->scale > 0.0f ? cfg->scale : (float)(1.0 / sqrt((double)L.D));
+    for (int i = 0; i < RECSA_MAX_C; ++i) tv.w[i] = i < cfg->C ? cfg->pooler_w[i] : 0.0f;
+    WorkView& wv = t->wv;
+    char* ws = (char*)workspace;
+    wv.status = (uint32_t*)(ws + L.o_status);
+    wv.lens = (int64_t*)(ws + L.o_lens);
+    wv.done = (uint32_t*)(ws + L.o_done);
+    wv.rope = (const float2*)(ws + L.o_rope);
+    wv.sel = (int32_t*)(ws + L.o_sel);
+    wv.cnt = (int32_t*)(ws + L.o_cnt);
+    wv.part = (float*)(ws + L.o_part);
+    wv.NL = L.NL;
+    wv.SPL = L.SPL;
+    wv.NS0 = L.NS0;
+    wv.NSLOT = L.NSLOT;
+    wv.ck = cfg->C * cfg->k;
+
+    cudaError_t e = prepare_kernels(cfg->dtype, L.D, L.G, L.SPL, L.NS0, cfg->C, cfg->k);
+    if (e == cudaSuccess) e = prepare_tree_kernels(tv, cfg->dtype);
+    if (e == cudaSuccess) e = launch_init_workspace(tv, wv, cfg->rope_base, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        free(t);
+        return RECSA_E_CUDA;
+    }
+    *out = t;
+    return RECSA_OK;
+}
+
+recsa_status recsa_build(recsa_tree* t, const int64_t* lengths, void* stream) {
+    if (!t || !lengths) return RECSA_E_INVAL;
+    for (int b = 0; b < t->B; ++b)
+        if (lengths[b] < 0 || lengths[b] > t->cap) return RECSA_E_CAPACITY;
+    cudaError_t e = launch_build(t->tv, t->wv, lengths, t->cfg.dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return RECSA_E_CUDA;
+    for (int b = 0; b < t->B; ++b) t->host_len[b] = lengths[b];
+    return RECSA_OK;
+}
+
+recsa_status recsa_append(recsa_tree* t, const void* k_new, const void* v_new, int32_t n,
+                          void* stream) {
+    if (!t || !k_new || !v_new || n < 1) return RECSA_E_INVAL;
+    if (!aligned16(k_new) || !aligned16(v_new)) return RECSA_E_INVAL;
+    for (int b = 0; b < t->B; ++b)
+        if (t->host_len[b] + n > t->cap) return RECSA_E_CAPACITY;
+    cudaError_t e = launch_append(t->tv, t->wv, k_new, v_new, n, t->cfg.dtype, (cudaStream_t)stream,
+                                  &t->prof);
+    if (e != cudaSuccess) return RECSA_E_CUDA;
+    for (int b = 0; b < t->B; ++b) t->host_len[b] += n;
+    return RECSA_OK;
+}
+
+recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_out,
+                          int32_t* counts_out, void* stream) {
+    if (!t || !q || !out) return RECSA_E_INVAL;
+    if (!aligned16(q) || !aligned16(out)) return RECSA_E_INVAL;
+    QueryView qv = {};
+    qv.q = q;
+    qv.out = out;
+    qv.sel_out = sel_out;
+    qv.cnt_out = counts_out;
+    qv.mode = 0;
+    qv.n_per_b = 1;
+    qv.pos0 = 0;
+    qv.q_begin = 0;
+    qv.nq = t->B;
+    return cuda_status(
+        launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof));
+}
+
+recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int32_t n, void* O,
+                                 int32_t* sel_out, int32_t* counts_out, void* stream) {
+    if (!t || !Q || !O || n < 1 || pos0 < 0) return RECSA_E_INVAL;
+    if (!aligned16(Q) || !aligned16(O)) return RECSA_E_INVAL;
+    for (int b = 0; b < t->B; ++b)
+        if (pos0 + n > t->host_len[b]) return RECSA_E_CAPACITY;
+    const int total = t->B * n;
+    for (int q0 = 0; q0 < total; q0 += t->Qmax) {
+        QueryView qv = {};
+        qv.q = Q;
+        qv.out = O;
+        qv.sel_out = sel_out;
+        qv.cnt_out = counts_out;
+        qv.mode = 1;
+        qv.n_per_b = n;
+        qv.pos0 = pos0;
+        qv.q_begin = q0;
+        qv.nq = total - q0 < t->Qmax ? total - q0 : t->Qmax;
+        cudaError_t e =
+            launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof);
+        if (e != cudaSuccess) return RECSA_E_CUDA;
+    }
+    return RECSA_OK;
+}
+
+recsa_status recsa_get_status(recsa_tree* t, void* stream) {
+    if (!t) return RECSA_E_INVAL;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RECSA_E_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, t->wv.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return RECSA_E_CUDA;
+    if (v != 0 && cudaMemset(t->wv.status, 0, sizeof(v)) != cudaSuccess) return RECSA_E_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return RECSA_E_CUDA;
+    switch (v) {
+        case kStatusOk: return RECSA_OK;
+        case kStatusCapacity: return RECSA_E_CAPACITY;
+        case kStatusTimeout: return RECSA_E_TIMEOUT;
+        default: return RECSA_E_DEVICE;
+    }
+}
+
+recsa_status recsa_tree_info(const recsa_tree* t, recsa_tree_info_t* info) {
+    if (!t || !info) return RECSA_E_INVAL;
+    info->n_levels = t->L.n_levels;
+    info->n_sel_levels = t->L.NL;
+    info->splits = t->L.SPL;
+    info->splits0 = t->L.NS0;
+    info->capacity = t->cap;
+    info->batch = t->B;
+    info->max_queries = t->Qmax;
+    return RECSA_OK;
+}
+
+recsa_status recsa_level_info(const recsa_tree* t, int32_t level, int64_t* k_offset,
+                              int64_t* v_offset, int64_t* rows) {
+    if (!t || level < 1 || level >= t->L.n_levels) return RECSA_E_INVAL;
+    if (k_offset) *k_offset = t->L.off_k[level];
+    if (v_offset) *v_offset = t->L.off_v[level];
+    if (rows) *rows = t->L.rows[level];
+    return RECSA_OK;
+}
+
+recsa_status recsa_host_lengths(const recsa_tree* t, int64_t* lengths) {
+    if (!t || !lengths) return RECSA_E_INVAL;
+    for (int b = 0; b < t->B; ++b) lengths[b] = t->host_len[b];
+    return RECSA_OK;
+}
+
+recsa_status recsa_set_profile_events(recsa_tree* t, int32_t which, void* start, void* stop) {
+    if (!t || ((start == nullptr) != (stop == nullptr))) return RECSA_E_INVAL;
+    if (start != nullptr && (which < -2 || which > t->L.NL)) return RECSA_E_INVAL;
+    t->prof.which = start ? which : -100;
+    t->prof.start = (cudaEvent_t)start;
+    t->prof.stop = (cudaEvent_t)stop;
+    return RECSA_OK;
+}
+
+recsa_status recsa_tree_free(recsa_tree* t) {
+    if (!t) return RECSA_E_INVAL;
+    free(t);
+    return RECSA_OK;
+}
+
+}  // extern "C"

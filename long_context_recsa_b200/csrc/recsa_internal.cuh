@@ -1,0 +1,234 @@
+// Internal declarations shared by the RecSA CUDA translation units (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/recsa.h"
+
+namespace recsa {
+
+constexpr int kMaxLevels = RECSA_MAX_LEVELS;
+constexpr int kThreads = 256;        // threads per CTA of the select/attend kernels
+constexpr int kWarps = kThreads / 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Device status word values (first error wins).
+enum : uint32_t { kStatusOk = 0, kStatusBadQuery = 1, kStatusCapacity = 2, kStatusTimeout = 3 };
+
+// Location of the tree in device memory.
+struct TreeView {
+    const void* k0;            // level 0 (caller's KV cache)
+    const void* v0;
+    void* k0w;                 // same pointers, writable (append)
+    void* v0w;
+    int64_t s_b, s_h, s_t;     // level-0 element strides
+    char* levels;              // level tables base
+    int64_t off_k[kMaxLevels]; // byte offsets of level l tables (l >= 1)
+    int64_t off_v[kMaxLevels];
+    int64_t rows[kMaxLevels];  // rows per (b, h) of level l (l >= 1); rows[0] = capacity
+    int B, Hkv, Hq, G, D, C, k;
+    int n_levels;              // stored levels at capacity, level 0 included
+    int64_t cap;
+    float scale;
+    float w[RECSA_MAX_C];      // pooler logits; kernels form softmax(w[0..m-1]) in fp64
+};
+
+// Which queries a select/attend launch handles.
+struct QueryView {
+    const void* q;             // [Qtot][Hq][D]
+    void* out;                 // [Qtot][Hq][D]
+    int32_t* sel_out;          // optional [Qtot][Hkv][NL][k]
+    int32_t* cnt_out;          // optional [Qtot][Hkv][NL+1]
+    int mode;                  // 0: decode (t = len-1); 1: prefill (t = pos0 + i)
+    int n_per_b;               // queries per sequence (1 for decode)
+    int64_t pos0;
+    int q_begin;               // first global query index of this wave
+    int nq;                    // queries in this wave
+};
+
+// Workspace carve-up.
+struct WorkView {
+    uint32_t* status;
+    int64_t* lens;             // [B] device-side lengths
+    uint32_t* done;            // [B] completion counters (append)
+    const float2* rope;        // [C*k][D/2] (cos, sin)
+    int32_t* sel;              // [Qmax][Hkv][NL][k]
+    int32_t* cnt;              // [Qmax][Hkv][NL+1]
+    float* part;               // [Qmax][Hkv][NSLOT][G][D+2]
+    int NL, SPL, NS0, NSLOT;
+    int ck;                    // C*k: rows of the RoPE table
+};
+
+// ----------------------------------------------------------------------------
+// small device helpers
+// ----------------------------------------------------------------------------
+
+__device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ void set_status(uint32_t* st, uint32_t code) {
+    atomicCAS(st, 0u, code);
+}
+
+template <typename T> struct VecOf;
+template <> struct VecOf<float> { static constexpr int N = 4; };
+template <> struct VecOf<__nv_bfloat16> { static constexpr int N = 8; };
+
+// Load 16 bytes (VecOf<T>::N elements) and widen to fp32.
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float* out);
+
+template <>
+__device__ __forceinline__ void load16<float>(const float* p, float* out) {
+    float4 v = *reinterpret_cast<const float4*>(p);
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, float* out) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = __uint_as_float(w[i] << 16);
+        out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Read-only path (data not written by the running kernel).
+template <typename T>
+__device__ __forceinline__ void load16_nc(const T* p, float* out);
+template <>
+__device__ __forceinline__ void load16_nc<float>(const float* p, float* out) {
+    float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load16_nc<__nv_bfloat16>(const __nv_bfloat16* p, float* out) {
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = __uint_as_float(w[i] << 16);
+        out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// fp64 -> storage rounding (round to nearest, ties to even), single rounding.
+__device__ __forceinline__ float round_store_f32(double x) { return __double2float_rn(x); }
+
+// fp64 -> bf16 with one correct rounding: round to odd at fp32 (24 bits, at least
+// two more than bf16's 8) and then to nearest even at bf16.  Rounding to odd first
+// makes the second rounding equal to a direct rounding of x (Boldo & Melquiond,
+// "Emulation of FMA and correctly rounded sums: proved algorithms using rounding
+// to odd", IEEE TC 2008).
+__device__ __forceinline__ __nv_bfloat16 round_store_bf16(double x) {
+    float f = __double2float_rz(x);
+    if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __float2bfloat16_rn(f);
+}
+
+template <typename T> __device__ __forceinline__ T store_round(double x);
+template <> __device__ __forceinline__ float store_round<float>(double x) { return round_store_f32(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 store_round<__nv_bfloat16>(double x) {
+    return round_store_bf16(x);
+}
+template <typename T> __device__ __forceinline__ T store_round_f(float x);
+template <> __device__ __forceinline__ float store_round_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 store_round_f<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Row pointers.
+template <typename T>
+__device__ __forceinline__ const T* level0_row(const TreeView& tv, int b, int h, int64_t t) {
+    return reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + h * tv.s_h + t * tv.s_t);
+}
+template <typename T>
+__device__ __forceinline__ const T* level0_vrow(const TreeView& tv, int b, int h, int64_t t) {
+    return reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + h * tv.s_h + t * tv.s_t);
+}
+template <typename T>
+__device__ __forceinline__ T* level_k(const TreeView& tv, int l, int b, int h) {
+    return reinterpret_cast<T*>(tv.levels + tv.off_k[l]) + ((int64_t)(b * tv.Hkv + h) * tv.rows[l]) * tv.D;
+}
+template <typename T>
+__device__ __forceinline__ T* level_v(const TreeView& tv, int l, int b, int h) {
+    return reinterpret_cast<T*>(tv.levels + tv.off_v[l]) + ((int64_t)(b * tv.Hkv + h) * tv.rows[l]) * tv.D;
+}
+
+// Query position of a (wave-local) query; returns false if it has nothing to do.
+__device__ __forceinline__ bool query_pos(const QueryView& qv, const WorkView& wv, int qloc,
+                                          int& b, int64_t& t, int& gq) {
+    gq = qv.q_begin + qloc;
+    b = gq / qv.n_per_b;
+    int i = gq - b * qv.n_per_b;
+    int64_t len = wv.lens[b];
+    t = (qv.mode == 0) ? len - 1 : qv.pos0 + i;
+    return t >= 0 && t < len;
+}
+
+// a^(l) = floor(t / C^l) for l = 0..; returns the first scored level l* (0 if none):
+// the highest l >= 1 whose full list [0..a^(l)] has more than k entries.
+__device__ __forceinline__ int first_scored_level(int64_t t, int C, int k, int64_t* a) {
+    int lstar = 0;
+    a[0] = t;
+    int l = 0;
+    int64_t p = t;
+    while (p > 0 && l + 1 < kMaxLevels) {
+        p /= C;
+        ++l;
+        a[l] = p;
+        if (p >= k) lstar = l;
+    }
+    for (int r = l + 1; r < kMaxLevels; ++r) a[r] = 0;
+    return lstar;
+}
+
+// |A^(level)| for a query whose first scored level is lstar >= level (Eq.3 sizes:
+// the list of l* is [0..a^(l*)], each lower list holds the C children of the
+// min(k, |A|) - 1 selected non-current nodes plus the current node's clamped
+// children).
+__device__ __forceinline__ int list_size(const int64_t* a, int lstar, int level, int C, int k) {
+    if (lstar == 0) return (int)(a[0] + 1);
+    int nA = (int)(a[lstar] + 1);
+    for (int l = lstar; l > level; --l) {
+        int nS = nA < k ? nA : k;
+        nA = C * (nS - 1) + (int)(a[l - 1] - (int64_t)C * a[l] + 1);
+    }
+    return nA;
+}
+
+__device__ __forceinline__ uint32_t ordered_key(float x) {
+    if (x == 0.0f) x = 0.0f;   // +0 and -0 compare equal: one key
+    uint32_t u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Optional events recorded around one kernel (see recsa_set_profile_events).
+struct ProfHook {
+    int which = -100;
+    cudaEvent_t start = nullptr, stop = nullptr;
+};
+
+inline void prof_mark(const ProfHook* p, int which, bool before, cudaStream_t s) {
+    if (p == nullptr || p->which != which || p->start == nullptr) return;
+    cudaEventRecordWithFlags(before ? p->start : p->stop, s, cudaEventRecordExternal);
+}
+
+// ----------------------------------------------------------------------------
+// launchers (defined in the .cu files)
+// ----------------------------------------------------------------------------
+cudaError_t launch_init_workspace(const TreeView& tv, const WorkView& wv, double rope_base,
+                                  cudaStream_t s);
+cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
+                         int dtype, cudaStream_t s);
+cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
+                          const void* v_new, int n, int dtype, cudaStream_t s,
+                          const ProfHook* prof = nullptr);
+cudaError_t launch_select_attend(const TreeView& tv, const WorkView& wv, const QueryView& qv,
+                                 int dtype, cudaStream_t s, const ProfHook* prof = nullptr);
+cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype);
+cudaError_t prepare_kernels(int dtype, int D, int G, int SPL, int NS0, int C, int k);
+
+}  // namespace recsa

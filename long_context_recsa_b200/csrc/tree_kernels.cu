@@ -1,0 +1,448 @@
+// Tree construction (Eq.1 of "Recursive Sparse Attention", section "Tree
+// Construction") and incremental append, sm_100a.
+//
+// A level-l node i pools its children C*i .. min(C*i+C-1, n_{l-1}-1) of level l-1:
+//   K = sum_c alpha_c K_c, alpha = softmax(w) over the m present children (stand-in
+//       pooler shared by all levels and heads),
+//   V = (1/m) sum_c V_c.
+// Sums run in fp64 and are rounded once to the storage dtype; the next level pools
+// the rounded values.  Build and append share warp_pool_node, so an appended tree
+// is bitwise equal to a rebuilt one.
+#include "recsa_internal.cuh"
+
+namespace recsa {
+
+template <typename T, int D>
+struct PoolShape {
+    static constexpr int VEC = VecOf<T>::N;   // elements per 16-byte load
+    static constexpr int RPL = D / VEC;       // lanes per row
+    static constexpr int RPW = 32 / RPL;      // rows per warp instruction
+    static constexpr int MAXIT = (RECSA_MAX_C + RPW - 1) / RPW;
+};
+
+// softmax(w[0..m-1]) for every m = 1..C, fp64, into alpha[(m-1)*C + c].
+__device__ void fill_alpha(const float* w, int C, double* alpha) {
+    for (int idx = threadIdx.x; idx < C * C; idx += blockDim.x) {
+        int m = idx / C + 1, c = idx % C;
+        double v = 0.0;
+        if (c < m) {
+            double mx = (double)w[0];
+            for (int j = 1; j < m; ++j) mx = fmax(mx, (double)w[j]);
+            double sum = 0.0;
+            for (int j = 0; j < m; ++j) sum += exp((double)w[j] - mx);
+            v = exp((double)w[c] - mx) / sum;
+        }
+        alpha[idx] = v;
+    }
+}
+
+// One warp pools m children rows (row stride rs elements) into one parent.
+// Deterministic: each lane sums its rows in increasing order, then row groups are
+// combined by a fixed butterfly.  The rounded parent is written to (dk, dv) and,
+// when given, also to (dk2, dv2).
+template <typename T, int D>
+__device__ __forceinline__ void warp_pool_node(const T* sk, const T* sv, int64_t rs, int m,
+                                               const double* alpha_m, T* dk, T* dv, T* dk2,
+                                               T* dv2) {
+    using P = PoolShape<T, D>;
+    const int lane = threadIdx.x & 31;
+    const int c = lane % P::RPL, r0 = lane / P::RPL;
+    double ak[P::VEC], av[P::VEC];
+#pragma unroll
+    for (int e = 0; e < P::VEC; ++e) { ak[e] = 0.0; av[e] = 0.0; }
+#pragma unroll
+    for (int it = 0; it < P::MAXIT; ++it) {
+        const int r = r0 + it * P::RPW;
+        if (r < m) {
+            float kx[P::VEC], vx[P::VEC];
+            load16<T>(sk + r * rs + c * P::VEC, kx);
+            load16<T>(sv + r * rs + c * P::VEC, vx);
+            const double al = alpha_m[r];
+#pragma unroll
+            for (int e = 0; e < P::VEC; ++e) {
+                ak[e] = fma(al, (double)kx[e], ak[e]);
+                av[e] += (double)vx[e];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = P::RPL; o < 32; o <<= 1) {
+#pragma unroll
+        for (int e = 0; e < P::VEC; ++e) {
+            ak[e] += __shfl_xor_sync(kFull, ak[e], o);
+            av[e] += __shfl_xor_sync(kFull, av[e], o);
+        }
+    }
+    if (r0 == 0) {
+        const double dm = (double)m;
+        union { uint4 u; T e[P::VEC]; } ok, ov;
+#pragma unroll
+        for (int e = 0; e < P::VEC; ++e) {
+            ok.e[e] = store_round<T>(ak[e]);
+            ov.e[e] = store_round<T>(av[e] / dm);
+        }
+        *reinterpret_cast<uint4*>(dk + c * P::VEC) = ok.u;
+        *reinterpret_cast<uint4*>(dv + c * P::VEC) = ov.u;
+        if (dk2 != nullptr) {
+            *reinterpret_cast<uint4*>(dk2 + c * P::VEC) = ok.u;
+            *reinterpret_cast<uint4*>(dv2 + c * P::VEC) = ov.u;
+        }
+    }
+}
+
+__device__ __forceinline__ int64_t ceil_div_pow(int64_t n, int C, int l) {
+    for (int i = 0; i < l; ++i) n = (n + C - 1) / C;
+    return n;
+}
+
+template <typename T>
+__device__ __forceinline__ void level_rows(const TreeView& tv, int l, int b, int h, const T*& k,
+                                           const T*& v, int64_t& rs) {
+    if (l == 0) {
+        k = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + h * tv.s_h);
+        v = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + h * tv.s_h);
+        rs = tv.s_t;
+    } else {
+        k = level_k<T>(tv, l, b, h);
+        v = level_v<T>(tv, l, b, h);
+        rs = tv.D;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// workspace initialisation: status, lengths, RoPE table
+// ----------------------------------------------------------------------------
+__global__ void init_workspace_kernel(WorkView wv, int B, int D, double base) {
+    const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gid == 0) *wv.status = 0u;
+    if (gid < B) { wv.lens[gid] = 0; wv.done[gid] = 0u; }
+    const int half = D / 2;
+    const int64_t total = (int64_t)wv.ck * half;
+    for (int64_t i = gid; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int p = (int)(i / half), j = (int)(i % half);
+        const double theta = pow(base, -2.0 * (double)j / (double)D);
+        const double ang = (double)p * theta;
+        float2 cs;
+        cs.x = (float)cos(ang);
+        cs.y = (float)sin(ang);
+        const_cast<float2*>(wv.rope)[i] = cs;
+    }
+}
+
+cudaError_t launch_init_workspace(const TreeView& tv, const WorkView& wv, double rope_base,
+                                  cudaStream_t s) {
+    const int64_t total = (int64_t)wv.ck * (tv.D / 2);
+    int blocks = (int)((total + 255) / 256);
+    if (blocks < 1) blocks = 1;
+    if (blocks > 4096) blocks = 4096;
+    init_workspace_kernel<<<blocks, 256, 0, s>>>(wv, tv.B, tv.D, rope_base);
+    return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// build passes: levels s+1 and s+2 from level s, over the nodes that cover a token
+// range.  add == 0: full rebuild of [0, len); add > 0: the tokens [len, len+add)
+// that an append has just written (len is the old length).
+// ----------------------------------------------------------------------------
+struct Lengths64 { int64_t v[RECSA_MAX_BATCH]; };
+
+__global__ void set_lengths_kernel(WorkView wv, Lengths64 L, int B) {
+    const int b = threadIdx.x;
+    if (b < B) wv.lens[b] = L.v[b];
+    if (b == 0) __threadfence();
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) build_pass_kernel(TreeView tv, WorkView wv, int s, int64_t add) {
+    __shared__ double alpha[RECSA_MAX_C * RECSA_MAX_C];
+    __shared__ float wsh[RECSA_MAX_C];
+    if (threadIdx.x < RECSA_MAX_C) wsh[threadIdx.x] = tv.w[threadIdx.x];
+    __syncthreads();
+    fill_alpha(wsh, tv.C, alpha);
+    __syncthreads();
+
+    const int bh = blockIdx.y;
+    const int b = bh / tv.Hkv, h = bh % tv.Hkv;
+    const int C = tv.C;
+    const int64_t len_old = wv.lens[b];
+    const int64_t L_new = len_old + add;
+    if (L_new > tv.cap || L_new <= 0) return;
+    const int64_t lo = (add == 0) ? 0 : len_old;
+    const int64_t hi = L_new;
+    const int64_t n_s = ceil_div_pow(L_new, C, s);
+    if (n_s <= 1) return;                         // level s is already the root
+    const int64_t n_s1 = (n_s + C - 1) / C;
+    const bool has_s2 = n_s1 > 1;
+    // level-(s+2) node range covering tokens [lo, hi)
+    int64_t span2 = 1;
+    for (int i = 0; i < s + 2; ++i) span2 *= C;
+    const int64_t p_lo = lo / span2, p_hi = (hi - 1) / span2;
+    const int warp = threadIdx.x >> 5;
+    const int64_t p2 = p_lo + (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (p2 > p_hi) return;
+
+    const T *sk, *sv;
+    int64_t rs;
+    level_rows<T>(tv, s, b, h, sk, sv, rs);
+    T* k1 = level_k<T>(tv, s + 1, b, h);
+    T* v1 = level_v<T>(tv, s + 1, b, h);
+    for (int c1 = 0; c1 < C; ++c1) {
+        const int64_t i1 = p2 * C + c1;
+        if (i1 >= n_s1) break;
+        const int m = (int)imin64(C, n_s - i1 * C);
+        warp_pool_node<T, D>(sk + i1 * C * rs, sv + i1 * C * rs, rs, m, alpha + (m - 1) * C,
+                             k1 + i1 * D, v1 + i1 * D, nullptr, nullptr);
+    }
+    if (has_s2) {
+        __syncwarp();
+        T* k2 = level_k<T>(tv, s + 2, b, h);
+        T* v2 = level_v<T>(tv, s + 2, b, h);
+        const int m = (int)imin64(C, n_s1 - p2 * C);
+        warp_pool_node<T, D>(k1 + p2 * C * D, v1 + p2 * C * D, D, m, alpha + (m - 1) * C,
+                             k2 + p2 * D, v2 + p2 * D, nullptr, nullptr);
+    }
+}
+
+// Copy n appended rows per (b, h) into level 0 at the current length.
+template <typename T, int D>
+__global__ void append_rows_kernel(TreeView tv, WorkView wv, const T* knew, const T* vnew, int n) {
+    const int bh = blockIdx.y;
+    const int b = bh / tv.Hkv, h = bh % tv.Hkv;
+    const int64_t L = wv.lens[b];
+    if (L + n > tv.cap) {
+        if (blockIdx.x == 0 && threadIdx.x == 0 && h == 0) set_status(wv.status, kStatusCapacity);
+        return;
+    }
+    constexpr int VEC = VecOf<T>::N;
+    constexpr int PER_ROW = D / VEC;
+    const int64_t total = (int64_t)n * PER_ROW;
+    T* k0 = reinterpret_cast<T*>(tv.k0w) + (b * tv.s_b + h * tv.s_h);
+    T* v0 = reinterpret_cast<T*>(tv.v0w) + (b * tv.s_b + h * tv.s_h);
+    const T* ks = knew + (int64_t)bh * n * D;
+    const T* vs = vnew + (int64_t)bh * n * D;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / PER_ROW, c = i % PER_ROW;
+        *reinterpret_cast<uint4*>(k0 + (L + r) * tv.s_t + c * VEC) =
+            *reinterpret_cast<const uint4*>(ks + r * D + c * VEC);
+        *reinterpret_cast<uint4*>(v0 + (L + r) * tv.s_t + c * VEC) =
+            *reinterpret_cast<const uint4*>(vs + r * D + c * VEC);
+    }
+}
+
+__global__ void commit_lengths_kernel(WorkView wv, int B, int64_t add, int64_t cap) {
+    const int b = threadIdx.x;
+    if (b < B && wv.lens[b] + add <= cap) wv.lens[b] += add;
+}
+
+// ----------------------------------------------------------------------------
+// single-token append: one CTA per (b, h) writes the token and re-pools its
+// ancestors bottom-up.  All unchanged siblings are staged in shared memory with one
+// round of loads; the chain then runs from shared memory.  The last CTA of a
+// sequence advances its length.
+// ----------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) append1_kernel(TreeView tv, WorkView wv, const T* knew,
+                                                      const T* vnew) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ double alpha[RECSA_MAX_C * RECSA_MAX_C];
+    __shared__ float wsh[RECSA_MAX_C];
+    __shared__ int lvl_m[kMaxLevels];
+    __shared__ int64_t lvl_i[kMaxLevels];
+    __shared__ int n_chain;
+    __shared__ bool is_last;
+
+    const int bh = blockIdx.x;
+    const int b = bh / tv.Hkv, h = bh % tv.Hkv;
+    const int C = tv.C;
+    const int64_t L = wv.lens[b];
+    if (L + 1 > tv.cap) {
+        if (threadIdx.x == 0 && h == 0) set_status(wv.status, kStatusCapacity);
+        return;
+    }
+    if (threadIdx.x < RECSA_MAX_C) wsh[threadIdx.x] = tv.w[threadIdx.x];
+    if (threadIdx.x == 0) {
+        // ancestors of token L: at level l the node L / C^l with m_l present children
+        int64_t n_prev = L + 1;                   // nodes at level l-1
+        int64_t idx = L;
+        int l = 1;
+        while (n_prev > 1 && l < kMaxLevels) {
+            const int64_t i = idx / C;
+            lvl_i[l] = i;
+            lvl_m[l] = (int)imin64(C, n_prev - i * C);
+            n_prev = (n_prev + C - 1) / C;
+            idx = i;
+            ++l;
+        }
+        n_chain = l - 1;                          // levels 1..n_chain change
+    }
+    __syncthreads();
+    fill_alpha(wsh, C, alpha);
+
+    // staging: slot l holds the C children rows (K then V) of the level-l ancestor
+    T* stage = reinterpret_cast<T*>(smem_raw);
+    const int64_t slot_elems = (int64_t)2 * C * D;
+    constexpr int VEC = VecOf<T>::N;
+    const T* kn = knew + (int64_t)bh * D;
+    const T* vn = vnew + (int64_t)bh * D;
+    T* k0 = reinterpret_cast<T*>(tv.k0w) + (b * tv.s_b + h * tv.s_h);
+    T* v0 = reinterpret_cast<T*>(tv.v0w) + (b * tv.s_b + h * tv.s_h);
+    // the new token: level 0 (global) and its slot in level 1's children
+    for (int e = threadIdx.x; e < D / VEC; e += blockDim.x) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(kn + e * VEC);
+        const uint4 vv = *reinterpret_cast<const uint4*>(vn + e * VEC);
+        *reinterpret_cast<uint4*>(k0 + L * tv.s_t + e * VEC) = kv;
+        *reinterpret_cast<uint4*>(v0 + L * tv.s_t + e * VEC) = vv;
+        if (n_chain >= 1) {
+            const int mm = lvl_m[1];
+            *reinterpret_cast<uint4*>(stage + (int64_t)(mm - 1) * D + e * VEC) = kv;
+            *reinterpret_cast<uint4*>(stage + (int64_t)C * D + (int64_t)(mm - 1) * D + e * VEC) = vv;
+        }
+    }
+    // unchanged siblings of every ancestor
+    for (int l = 1; l <= n_chain; ++l) {
+        const T *sk, *sv;
+        int64_t rs;
+        level_rows<T>(tv, l - 1, b, h, sk, sv, rs);
+        const int m = lvl_m[l];
+        const int64_t first = lvl_i[l] * C;
+        T* slot = stage + (int64_t)(l - 1) * slot_elems;
+        const int per_row = D / VEC;
+        for (int e = threadIdx.x; e < (m - 1) * per_row; e += blockDim.x) {
+            const int r = e / per_row, c = e % per_row;
+            *reinterpret_cast<uint4*>(slot + (int64_t)r * D + c * VEC) =
+                *reinterpret_cast<const uint4*>(sk + (first + r) * rs + c * VEC);
+            *reinterpret_cast<uint4*>(slot + (int64_t)C * D + (int64_t)r * D + c * VEC) =
+                *reinterpret_cast<const uint4*>(sv + (first + r) * rs + c * VEC);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        for (int l = 1; l <= n_chain; ++l) {
+            const int m = lvl_m[l];
+            const T* slot = stage + (int64_t)(l - 1) * slot_elems;
+            T* nk = nullptr;
+            T* nv = nullptr;
+            if (l < n_chain) {                     // the new node is the last child above
+                T* up = stage + (int64_t)l * slot_elems;
+                const int mu = lvl_m[l + 1];
+                nk = up + (int64_t)(mu - 1) * D;
+                nv = up + (int64_t)C * D + (int64_t)(mu - 1) * D;
+            }
+            warp_pool_node<T, D>(slot, slot + (int64_t)C * D, D, m, alpha + (m - 1) * C,
+                                 level_k<T>(tv, l, b, h) + lvl_i[l] * D,
+                                 level_v<T>(tv, l, b, h) + lvl_i[l] * D, nk, nv);
+            __syncwarp();
+        }
+    }
+    // advance the length once every head of this sequence is done
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&wv.done[b], 1u);
+        is_last = (prev == (unsigned)tv.Hkv - 1);
+    }
+    __syncthreads();
+    if (is_last && threadIdx.x == 0) {
+        __threadfence();
+        wv.lens[b] = L + 1;
+        wv.done[b] = 0u;
+        __threadfence();
+    }
+}
+
+// ----------------------------------------------------------------------------
+// host launchers
+// ----------------------------------------------------------------------------
+template <typename T, int D>
+static cudaError_t run_passes(const TreeView& tv, const WorkView& wv, int64_t add, cudaStream_t s) {
+    for (int src = 0; src + 1 < tv.n_levels; src += 2) {
+        int64_t span2 = 1;
+        for (int i = 0; i < src + 2; ++i) span2 *= tv.C;
+        const int64_t tokens = (add == 0) ? tv.cap : add;
+        const int64_t nodes = (tokens + span2 - 1) / span2 + 1;
+        const int64_t blocks = (nodes + 7) / 8;
+        dim3 grid((unsigned)blocks, (unsigned)(tv.B * tv.Hkv));
+        build_pass_kernel<T, D><<<grid, 256, 0, s>>>(tv, wv, src, add);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <typename T, int D>
+static cudaError_t build_impl(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
+                              cudaStream_t s) {
+    Lengths64 L{};
+    for (int b = 0; b < tv.B; ++b) L.v[b] = lengths[b];
+    set_lengths_kernel<<<1, RECSA_MAX_BATCH, 0, s>>>(wv, L, tv.B);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return run_passes<T, D>(tv, wv, 0, s);
+}
+
+constexpr size_t kAppend1MaxSmem = 160 * 1024;
+
+static size_t append1_smem(const TreeView& tv, int esize) {
+    return (size_t)(tv.n_levels) * 2 * tv.C * tv.D * esize;
+}
+
+template <typename T, int D>
+static cudaError_t append_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
+                               const void* v_new, int n, cudaStream_t s, const ProfHook* prof) {
+    const size_t sm = append1_smem(tv, (int)sizeof(T));
+    if (n == 1 && sm <= kAppend1MaxSmem) {
+        prof_mark(prof, -1, true, s);
+        append1_kernel<T, D><<<tv.B * tv.Hkv, 128, sm, s>>>(
+            tv, wv, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new));
+        prof_mark(prof, -1, false, s);
+        return cudaGetLastError();
+    }
+    const int per_row = D / VecOf<T>::N;
+    int64_t blocks = ((int64_t)n * per_row + 255) / 256;
+    if (blocks > 1024) blocks = 1024;
+    prof_mark(prof, -1, true, s);
+    append_rows_kernel<T, D><<<dim3((unsigned)blocks, tv.B * tv.Hkv), 256, 0, s>>>(
+        tv, wv, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new), n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = run_passes<T, D>(tv, wv, n, s);
+    if (e != cudaSuccess) return e;
+    commit_lengths_kernel<<<1, RECSA_MAX_BATCH, 0, s>>>(wv, tv.B, n, tv.cap);
+    prof_mark(prof, -1, false, s);
+    return cudaGetLastError();
+}
+
+#define RECSA_DISPATCH_TD(dtype, D, FN, ...)                                              \
+    do {                                                                                  \
+        if ((dtype) == RECSA_BF16 && (D) == 128) return FN<__nv_bfloat16, 128>(__VA_ARGS__); \
+        if ((dtype) == RECSA_BF16 && (D) == 64) return FN<__nv_bfloat16, 64>(__VA_ARGS__);   \
+        if ((dtype) == RECSA_F32 && (D) == 128) return FN<float, 128>(__VA_ARGS__);          \
+        if ((dtype) == RECSA_F32 && (D) == 64) return FN<float, 64>(__VA_ARGS__);            \
+        return cudaErrorInvalidValue;                                                     \
+    } while (0)
+
+template <typename T, int D>
+static cudaError_t prepare_tree_impl(const TreeView& tv) {
+    const size_t sm = append1_smem(tv, (int)sizeof(T));
+    if (sm > kAppend1MaxSmem) return cudaSuccess;     // multi-pass path is used instead
+    return cudaFuncSetAttribute(append1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sm);
+}
+
+cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype) {
+    RECSA_DISPATCH_TD(dtype, tv.D, prepare_tree_impl, tv);
+}
+
+cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
+                         int dtype, cudaStream_t s) {
+    RECSA_DISPATCH_TD(dtype, tv.D, build_impl, tv, wv, lengths, s);
+}
+
+cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
+                          const void* v_new, int n, int dtype, cudaStream_t s,
+                          const ProfHook* prof) {
+    RECSA_DISPATCH_TD(dtype, tv.D, append_impl, tv, wv, k_new, v_new, n, s, prof);
+}
+
+}  // namespace recsa

@@ -1,0 +1,201 @@
+"""GPU parity: librecsa.so (through its C ABI) against the fp64 oracle.
+
+Tree tables bit-exact; selected sets bit-exact except at stated near-ties (the
+(k-1)-th and k-th importances within 1e-5 relative); attention outputs within
+2e-2 max-abs for bf16 and 1e-5 for fp32.
+"""
+import numpy as np
+import pytest
+import torch
+
+from tests import parity_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def R():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_recsa_b200 import build
+    build.build()
+    import long_context_recsa_b200.recsa as R
+    return R
+
+
+def run_decode_case(R, *, config_id, B, Hkv, Hq, d, C, k, lengths, dtype, cap=None,
+                    n_needles=0, base=1e6, check_units=None, check_tree=True):
+    cap = cap or max(lengths)
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype=dtype,
+                   rope_base=base, pooler_w=w)
+    K, V, q = H.make_inputs(config_id, B, Hkv, Hq, d, cap, lengths, dtype, n_needles=n_needles)
+    q = q[:, 0].contiguous()
+    tree = R.RecsaTree(cfg, cap, B, k0=K, v0=V)
+    tree.recsa_build(lengths)
+    out, sel, cnt = tree.decode(q, with_sel=True)
+    torch.cuda.synchronize()
+    assert tree.recsa_get_status() == R.RECSA_OK
+    G = Hq // Hkv
+    units = check_units or [(b, h) for b in range(B) for h in range(Hkv)]
+    worst = 0.0
+    for b, h in units:
+        L = lengths[b]
+        if L == 0:
+            assert torch.all(out[b] == 0)
+            continue
+        t = L - 1
+        levels, res = H.oracle_unit(K[b, h], V[b, h], q[b, h * G:(h + 1) * G], L, t, C, k, w,
+                                    dtype, base)
+        if check_tree:
+            H.compare_tree(tree, levels, b, h, dtype)
+        sel_u = sel[b, h].cpu().numpy() if tree.n_sel_levels else np.zeros((0, k))
+        cur = H.check_selection(levels, H.to64(q[b, h * G:(h + 1) * G]), t, C, k, base, res,
+                                sel_u, cnt[b, h].cpu().numpy(), tree.n_sel_levels)
+        err = H.max_abs(H.to64(out[b, h * G:(h + 1) * G]), cur.out)
+        worst = max(worst, err)
+        assert err <= H.TOL_OUT[dtype], f"unit {(b, h)}: output max-abs {err}"
+    return tree, worst
+
+
+def test_tiny_fp32_config(R):
+    """Tiny decode: 1 KV head, 2 query heads, d=64, L=4096, C=16, k=8, fp32."""
+    _, worst = run_decode_case(R, config_id=1, B=1, Hkv=1, Hq=2, d=64, C=16, k=8,
+                               lengths=[4096], dtype="f32")
+    print("tiny fp32 worst max-abs", worst)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("C,k,d,G", [(4, 3, 64, 2), (16, 8, 128, 4), (2, 5, 64, 1), (8, 16, 128, 8)])
+def test_small_ragged_batches(R, dtype, C, k, d, G):
+    Hkv = 2
+    lengths = [1000, 777, 64 * C + 1, 5]
+    run_decode_case(R, config_id=11, B=4, Hkv=Hkv, Hq=G * Hkv, d=d, C=C, k=k, lengths=lengths,
+                    dtype=dtype, cap=1100, n_needles=3)
+
+
+@pytest.mark.parametrize("L", [1, 2, 15, 16, 17, 255, 256, 257, 4095, 4096, 4097, 6000])
+def test_edge_lengths(R, L):
+    """Single token, exact powers of C, one past them, the dense regime (t < C*k,
+    nothing scored) and the first scored lengths."""
+    run_decode_case(R, config_id=12, B=1, Hkv=1, Hq=4, d=128, C=16, k=16, lengths=[L],
+                    dtype="bf16", cap=max(L, 16))
+
+
+def test_zero_length_sequence_outputs_zero(R):
+    run_decode_case(R, config_id=13, B=2, Hkv=1, Hq=2, d=64, C=4, k=2, lengths=[0, 50],
+                    dtype="f32", cap=64)
+
+
+def test_zero_query_tie_break(R):
+    """q = 0: all importances equal, TopK keeps the lowest indices (ties to the
+    lower index), identical on GPU and oracle."""
+    C, k, d, L = 4, 3, 64, 900
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=2, n_kv_heads=1, C=C, k=k, dtype="f32", pooler_w=w)
+    K, V, _ = H.make_inputs(14, 1, 1, 2, d, L, [L], "f32")
+    q = torch.zeros(1, 2, d, device="cuda")
+    tree = R.RecsaTree(cfg, L, 1, k0=K, v0=V)
+    tree.recsa_build([L])
+    out, sel, cnt = tree.decode(q, with_sel=True)
+    levels, res = H.oracle_unit(K[0, 0], V[0, 0], q[0], L, L - 1, C, k, w, "f32", 1e6)
+    for tr in res.levels:
+        if tr.scored:
+            np.testing.assert_array_equal(sel[0, 0, tr.level - 1].cpu().numpy(), tr.S)
+            np.testing.assert_array_equal(tr.S[:-1], tr.A[: k - 1])
+    assert H.max_abs(H.to64(out[0]), res.out) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_append_equals_build_bitwise(R, dtype):
+    """build(L) then append one token at a time (and a multi-token chunk) equals
+    build(L + n) bit for bit, tables and decode outputs."""
+    C, k, d, Hkv, Hq, B = 16, 8, 128, 2, 8, 2
+    L0, steps, chunk = 4000, 40, 300
+    cap = L0 + steps + chunk
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype=dtype, pooler_w=w)
+    K, V, q = H.make_inputs(15, B, Hkv, Hq, d, cap, [cap] * B, dtype)
+    q = q[:, 0].contiguous()
+    Ka = K.clone()
+    Va = V.clone()
+    Ka[:, :, L0:] = 0
+    Va[:, :, L0:] = 0
+    inc = R.RecsaTree(cfg, cap, B, k0=Ka, v0=Va)
+    inc.recsa_build([L0] * B)
+    outs_inc = []
+    for s in range(steps):
+        kn = K[:, :, L0 + s: L0 + s + 1].contiguous()
+        vn = V[:, :, L0 + s: L0 + s + 1].contiguous()
+        inc.recsa_append(kn, vn)
+        outs_inc.append(inc.decode(q)[0])
+    kn = K[:, :, L0 + steps:].contiguous()
+    vn = V[:, :, L0 + steps:].contiguous()
+    inc.recsa_append(kn, vn)
+    out_inc_final = inc.decode(q)[0]
+    torch.cuda.synchronize()
+    assert inc.recsa_get_status() == R.RECSA_OK
+    assert inc.host_lengths() == [cap] * B
+    full = R.RecsaTree(cfg, cap, B, k0=K.clone(), v0=V.clone())
+    full.recsa_build([cap] * B)
+    for l in range(1, full.n_levels):
+        Ki, Vi = inc.level_tables(l)
+        Kf, Vf = full.level_tables(l)
+        n = -(-cap // C ** l)
+        assert torch.equal(Ki[:, :, :n], Kf[:, :, :n]), f"K level {l}"
+        assert torch.equal(Vi[:, :, :n], Vf[:, :, :n]), f"V level {l}"
+    assert torch.equal(out_inc_final, full.decode(q)[0])
+    # intermediate steps against fresh builds at a few lengths
+    for s in (0, 7, steps - 1):
+        ref = R.RecsaTree(cfg, cap, B, k0=K.clone(), v0=V.clone())
+        ref.recsa_build([L0 + s + 1] * B)
+        assert torch.equal(outs_inc[s], ref.decode(q)[0]), f"step {s}"
+
+
+def test_prefill_rows_equal_decode_on_truncated_tree(R):
+    """Causality: prefill row t equals decode of a tree holding only [0..t]
+    (bitwise, same kernels), and matches the oracle."""
+    C, k, d, Hkv, Hq = 16, 8, 128, 2, 8
+    L = 5000
+    pos0, n = 4990, 10
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype="bf16", pooler_w=w)
+    K, V, Q = H.make_inputs(16, 1, Hkv, Hq, d, L, [L], "bf16", q_rows=n, n_needles=5)
+    tree = R.RecsaTree(cfg, L, 1, max_queries=8, k0=K, v0=V)
+    tree.recsa_build([L])
+    O, sel, cnt = tree.prefill(Q, pos0, with_sel=True)
+    torch.cuda.synchronize()
+    assert tree.recsa_get_status() == R.RECSA_OK
+    G = Hq // Hkv
+    for i in range(n):
+        t = pos0 + i
+        trunc = R.RecsaTree(cfg, L, 1, k0=K.clone(), v0=V.clone())
+        trunc.recsa_build([t + 1])
+        od, sd, cd = trunc.decode(Q[:, i].contiguous(), with_sel=True)
+        assert torch.equal(O[:, i], od), f"row {i}"
+        assert torch.equal(sel[i], sd[0]) and torch.equal(cnt[i], cd[0])
+        for h in range(Hkv):
+            levels, res = H.oracle_unit(K[0, h], V[0, h], Q[0, i, h * G:(h + 1) * G], L, t, C, k,
+                                        w, "bf16", 1e6)
+            cur = H.check_selection(levels, H.to64(Q[0, i, h * G:(h + 1) * G]), t, C, k, 1e6, res,
+                                    sel[i, h].cpu().numpy(), cnt[i, h].cpu().numpy(),
+                                    tree.n_sel_levels)
+            assert H.max_abs(H.to64(O[0, i, h * G:(h + 1) * G]), cur.out) <= 2e-2
+
+
+def test_host_errors_are_returned_not_launched(R):
+    cfg = R.Config(head_dim=64, n_q_heads=2, n_kv_heads=1, C=4, k=2, dtype="f32",
+                   pooler_w=H.w_for(4))
+    tree = R.RecsaTree(cfg, 100, 1)
+    tree.recsa_build([90])
+    kn = torch.zeros(1, 1, 20, 64, device="cuda")
+    with pytest.raises(R.RecsaError) as e:
+        tree.recsa_append(kn, kn)
+    assert e.value.status == R.RECSA_E_CAPACITY
+    with pytest.raises(R.RecsaError) as e:
+        tree.recsa_build([101])
+    assert e.value.status == R.RECSA_E_CAPACITY
+    Q = torch.zeros(1, 5, 2, 64, device="cuda")
+    with pytest.raises(R.RecsaError):
+        tree.prefill(Q, 88)
+    assert tree.recsa_get_status() == R.RECSA_OK
