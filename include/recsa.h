@@ -194,6 +194,31 @@ RECSA_API recsa_status recsa_host_lengths(const recsa_tree* tree, int64_t* lengt
 RECSA_API recsa_status recsa_set_profile_events(recsa_tree* tree, int32_t which, void* start,
                                                 void* stop);
 
+/* Decode without any device allocation by the caller or the library.  The paper
+ * has no counterpart to this call; it exists for callers that cannot allocate device
+ * memory where they call decode (inside a stream capture in global capture mode, in
+ * a loop bound to a fixed pre-planned memory budget, or in a runtime with no device
+ * allocator for per-call scratch) and so cannot provide recsa_decode's workspace.
+ * Same result as recsa_decode on a tree with these buffers and lengths.
+ *   cfg, capacity, batch   as for recsa_tree_init (one query per sequence).
+ *   k0, v0, kv_strides     level-0 cache, as for recsa_tree_init.
+ *   levels, level_bytes    level tables already built by recsa_build/recsa_append
+ *                          for these lengths, laid out as recsa_query_sizes states.
+ *   lengths                host array [batch]; query b sits at lengths[b] - 1.
+ *   q, out                 [batch][Hq][d] device, 16-byte aligned.
+ * Scratch: a fixed 8 MiB device array inside the library (held by every GPU that
+ * loads it until exit), shared by all calls: calls that may overlap on the GPU race.
+ * A shape whose workspace (recsa_query_sizes with max_queries = batch) exceeds 8 MiB
+ * is rejected with RECSA_E_CAPACITY.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  No cudaMalloc, cudaFree or allocating library
+ * routine is called. */
+RECSA_API recsa_status recsa_decode_noalloc(const recsa_config* cfg, int64_t capacity,
+                                            int32_t batch, const void* k0, const void* v0,
+                                            const int64_t kv_strides[3], const void* levels,
+                                            size_t level_bytes, const int64_t* lengths,
+                                            const void* q, void* out, void* stream);
+
 /* Free the host handle.  Device memory stays with the caller. */
 RECSA_API recsa_status recsa_tree_free(recsa_tree* tree);
 

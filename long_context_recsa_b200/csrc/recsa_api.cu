@@ -94,6 +94,61 @@ static recsa_status compute_layout(const recsa_config* c, int64_t cap, int B, in
     return RECSA_OK;
 }
 
+// Tree and workspace views over caller buffers and a scratch base `ws`, without a
+// tree handle (used by recsa_decode_noalloc).  Same layout as recsa_tree_init.
+// With ws == nullptr only *ws_bytes is computed.
+recsa_status views_for(const recsa_config* cfg, int64_t cap, int B, int Qmax, const void* k0,
+                       const void* v0, const int64_t strides[3], const void* levels,
+                       size_t level_bytes, char* ws, size_t* ws_bytes, TreeView* tv,
+                       WorkView* wv) {
+    Layout L;
+    recsa_status st = compute_layout(cfg, cap, B, Qmax, &L);
+    if (st != RECSA_OK) return st;
+    *ws_bytes = L.ws_bytes;
+    if (ws == nullptr) return RECSA_OK;
+    if (!k0 || !v0 || !strides || !levels) return RECSA_E_INVAL;
+    if ((((uintptr_t)k0) & 15u) || (((uintptr_t)v0) & 15u) || (((uintptr_t)levels) & 255u))
+        return RECSA_E_INVAL;
+    const int64_t per16 = 16 / L.esize;
+    if (strides[0] < 0 || strides[1] < 0 || strides[2] < L.D) return RECSA_E_INVAL;
+    if (strides[0] % per16 || strides[1] % per16 || strides[2] % per16) return RECSA_E_INVAL;
+    if (level_bytes < L.level_bytes) return RECSA_E_CAPACITY;
+    memset(tv, 0, sizeof(*tv));
+    memset(wv, 0, sizeof(*wv));
+    tv->k0 = k0; tv->v0 = v0; tv->k0w = nullptr; tv->v0w = nullptr;
+    tv->s_b = strides[0]; tv->s_h = strides[1]; tv->s_t = strides[2];
+    tv->levels = (char*)levels;
+    for (int l = 0; l < kMaxLevels; ++l) {
+        tv->off_k[l] = L.off_k[l];
+        tv->off_v[l] = L.off_v[l];
+        tv->rows[l] = L.rows[l];
+    }
+    tv->B = B;
+    tv->Hkv = cfg->n_kv_heads;
+    tv->Hq = cfg->n_q_heads;
+    tv->G = L.G;
+    tv->D = L.D;
+    tv->C = cfg->C;
+    tv->k = cfg->k;
+    tv->n_levels = L.n_levels;
+    tv->cap = cap;
+    tv->scale = cfg->scale > 0.0f ? cfg->scale : (float)(1.0 / sqrt((double)L.D));
+    for (int i = 0; i < RECSA_MAX_C; ++i) tv->w[i] = i < cfg->C ? cfg->pooler_w[i] : 0.0f;
+    wv->status = (uint32_t*)(ws + L.o_status);
+    wv->lens = (int64_t*)(ws + L.o_lens);
+    wv->done = (uint32_t*)(ws + L.o_done);
+    wv->rope = (const float2*)(ws + L.o_rope);
+    wv->sel = (int32_t*)(ws + L.o_sel);
+    wv->cnt = (int32_t*)(ws + L.o_cnt);
+    wv->part = (float*)(ws + L.o_part);
+    wv->NL = L.NL;
+    wv->SPL = L.SPL;
+    wv->NS0 = L.NS0;
+    wv->NSLOT = L.NSLOT;
+    wv->ck = cfg->C * cfg->k;
+    return RECSA_OK;
+}
+
 }  // namespace recsa
 
 using namespace recsa;

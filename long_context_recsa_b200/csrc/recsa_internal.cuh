@@ -229,6 +229,11 @@ cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_
 cudaError_t launch_select_attend(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                  int dtype, cudaStream_t s, const ProfHook* prof = nullptr);
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype);
+cudaError_t launch_set_lengths(const WorkView& wv, const int64_t* lengths, int B, cudaStream_t s);
+recsa_status views_for(const recsa_config* cfg, int64_t cap, int B, int Qmax, const void* k0,
+                       const void* v0, const int64_t strides[3], const void* levels,
+                       size_t level_bytes, char* ws, size_t* ws_bytes, TreeView* tv,
+                       WorkView* wv);
 cudaError_t prepare_kernels(int dtype, int D, int G, int SPL, int NS0, int C, int k);
 
 }  // namespace recsa

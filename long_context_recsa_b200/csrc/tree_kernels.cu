@@ -434,6 +434,13 @@ cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype) {
     RECSA_DISPATCH_TD(dtype, tv.D, prepare_tree_impl, tv);
 }
 
+cudaError_t launch_set_lengths(const WorkView& wv, const int64_t* lengths, int B, cudaStream_t s) {
+    Lengths64 L{};
+    for (int b = 0; b < B; ++b) L.v[b] = lengths[b];
+    set_lengths_kernel<<<1, RECSA_MAX_BATCH, 0, s>>>(wv, L, B);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
                          int dtype, cudaStream_t s) {
     RECSA_DISPATCH_TD(dtype, tv.D, build_impl, tv, wv, lengths, s);
