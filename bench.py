@@ -42,6 +42,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--batch", type=int, default=4,
+                   help="sequences per GPU (the headline workload uses 4)")
     return p.parse_args()
 
 
@@ -160,6 +163,7 @@ def barrier(ws):
 
 def run_ours(args):
     import torch
+    W["B"] = args.batch
     from long_context_recsa_b200 import build, inputs as I
     build.build()
     import long_context_recsa_b200.recsa as R
@@ -285,7 +289,7 @@ def run_ours(args):
         res["e2e"] = e2e_decode(tree, R, knew, vnew, qs, args, ws, flush)
     if not args.no_prefill:
         res["prefill"] = bench_prefill(R, I, cfg, K, V, tree, args, ws, dev, flush)
-    if rank == 0:
+    if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(K, V, qs, cfg, R)
     if ws > 1:
         import torch.distributed as dist

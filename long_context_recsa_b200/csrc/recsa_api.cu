@@ -17,7 +17,7 @@ struct Layout {
     int64_t off_k[kMaxLevels], off_v[kMaxLevels];
     size_t level_bytes;
     int NL, SPL, NS0, NSLOT;
-    size_t o_status, o_lens, o_done, o_rope, o_sel, o_cnt, o_part, ws_bytes;
+    size_t o_status, o_lens, o_done, o_alpha, o_rope, o_sel, o_cnt, o_part, o_ucnt, ws_bytes;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -86,10 +86,12 @@ static recsa_status compute_layout(const recsa_config* c, int64_t cap, int B, in
     L->o_status = w; w = al256(w + 64);
     L->o_lens = w;   w = al256(w + sizeof(int64_t) * B);
     L->o_done = w;   w = al256(w + sizeof(uint32_t) * B);
+    L->o_alpha = w;  w = al256(w + sizeof(double) * RECSA_MAX_C * RECSA_MAX_C);
     L->o_rope = w;   w = al256(w + sizeof(float2) * (size_t)ck * (L->D / 2));
     L->o_sel = w;    w = al256(w + sizeof(int32_t) * (size_t)Qmax * Hkv * (NL > 0 ? NL : 1) * c->k);
     L->o_cnt = w;    w = al256(w + sizeof(int32_t) * (size_t)Qmax * Hkv * (NL + 1));
     L->o_part = w;   w = al256(w + sizeof(float) * (size_t)Qmax * Hkv * L->NSLOT * L->G * (L->D + 2));
+    L->o_ucnt = w;   w = al256(w + sizeof(uint32_t) * (size_t)Qmax * Hkv);
     L->ws_bytes = w;
     return RECSA_OK;
 }
@@ -130,17 +132,22 @@ recsa_status views_for(const recsa_config* cfg, int64_t cap, int B, int Qmax, co
     tv->D = L.D;
     tv->C = cfg->C;
     tv->k = cfg->k;
+    tv->lgC = (cfg->C & (cfg->C - 1)) == 0 ? __builtin_ctz((unsigned)cfg->C) : -1;
     tv->n_levels = L.n_levels;
     tv->cap = cap;
     tv->scale = cfg->scale > 0.0f ? cfg->scale : (float)(1.0 / sqrt((double)L.D));
+    tv->rope_base = cfg->rope_base;
     for (int i = 0; i < RECSA_MAX_C; ++i) tv->w[i] = i < cfg->C ? cfg->pooler_w[i] : 0.0f;
     wv->status = (uint32_t*)(ws + L.o_status);
     wv->lens = (int64_t*)(ws + L.o_lens);
     wv->done = (uint32_t*)(ws + L.o_done);
+    wv->alpha = (const double*)(ws + L.o_alpha);
     wv->rope = (const float2*)(ws + L.o_rope);
     wv->sel = (int32_t*)(ws + L.o_sel);
     wv->cnt = (int32_t*)(ws + L.o_cnt);
     wv->part = (float*)(ws + L.o_part);
+    wv->ucnt = (uint32_t*)(ws + L.o_ucnt);
+    wv->nunits = Qmax * cfg->n_kv_heads;
     wv->NL = L.NL;
     wv->SPL = L.SPL;
     wv->NS0 = L.NS0;
@@ -236,19 +243,24 @@ recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t 
     tv.D = L.D;
     tv.C = cfg->C;
     tv.k = cfg->k;
+    tv.lgC = (cfg->C & (cfg->C - 1)) == 0 ? __builtin_ctz((unsigned)cfg->C) : -1;
     tv.n_levels = L.n_levels;
     tv.cap = capacity;
     tv.scale = cfg->scale > 0.0f ? cfg->scale : (float)(1.0 / sqrt((double)L.D));
+    tv.rope_base = cfg->rope_base;
     for (int i = 0; i < RECSA_MAX_C; ++i) tv.w[i] = i < cfg->C ? cfg->pooler_w[i] : 0.0f;
     WorkView& wv = t->wv;
     char* ws = (char*)workspace;
     wv.status = (uint32_t*)(ws + L.o_status);
     wv.lens = (int64_t*)(ws + L.o_lens);
     wv.done = (uint32_t*)(ws + L.o_done);
+    wv.alpha = (const double*)(ws + L.o_alpha);
     wv.rope = (const float2*)(ws + L.o_rope);
     wv.sel = (int32_t*)(ws + L.o_sel);
     wv.cnt = (int32_t*)(ws + L.o_cnt);
     wv.part = (float*)(ws + L.o_part);
+    wv.ucnt = (uint32_t*)(ws + L.o_ucnt);
+    wv.nunits = max_queries * cfg->n_kv_heads;
     wv.NL = L.NL;
     wv.SPL = L.SPL;
     wv.NS0 = L.NS0;

@@ -29,9 +29,11 @@ struct TreeView {
     int64_t off_v[kMaxLevels];
     int64_t rows[kMaxLevels];  // rows per (b, h) of level l (l >= 1); rows[0] = capacity
     int B, Hkv, Hq, G, D, C, k;
+    int lgC;                   // log2(C) when C is a power of two, else -1
     int n_levels;              // stored levels at capacity, level 0 included
     int64_t cap;
     float scale;
+    double rope_base;
     float w[RECSA_MAX_C];      // pooler logits; kernels form softmax(w[0..m-1]) in fp64
 };
 
@@ -54,9 +56,12 @@ struct WorkView {
     int64_t* lens;             // [B] device-side lengths
     uint32_t* done;            // [B] completion counters (append)
     const float2* rope;        // [C*k][D/2] (cos, sin)
+    const double* alpha;       // [C][C]: alpha[(m-1)*C + c] = softmax(w[0..m-1])_c
     int32_t* sel;              // [Qmax][Hkv][NL][k]
     int32_t* cnt;              // [Qmax][Hkv][NL+1]
     float* part;               // [Qmax][Hkv][NSLOT][G][D+2]
+    uint32_t* ucnt;            // [Qmax*Hkv] level-0 CTAs finished per unit (reset to 0)
+    int nunits;                // Qmax*Hkv
     int NL, SPL, NS0, NSLOT;
     int ck;                    // C*k: rows of the RoPE table
 };
@@ -168,33 +173,47 @@ __device__ __forceinline__ bool query_pos(const QueryView& qv, const WorkView& w
     return t >= 0 && t < len;
 }
 
-// a^(l) = floor(t / C^l) for l = 0..; returns the first scored level l* (0 if none):
-// the highest l >= 1 whose full list [0..a^(l)] has more than k entries.
-__device__ __forceinline__ int first_scored_level(int64_t t, int C, int k, int64_t* a) {
-    int lstar = 0;
-    a[0] = t;
-    int l = 0;
+// Division by the branching factor: a shift when C is a power of two.
+__device__ __forceinline__ int64_t cdiv64(int64_t x, int C, int lgC) { return lgC >= 0 ? (x >> lgC) : x / C; }
+__device__ __forceinline__ int cdiv(int x, int C, int lgC) { return lgC >= 0 ? (x >> lgC) : x / C; }
+__device__ __forceinline__ int cmod(int x, int C, int lgC) { return lgC >= 0 ? (x & (C - 1)) : x % C; }
+
+// a^(l) = floor(t / C^l).
+__device__ __forceinline__ int64_t apow(int64_t t, int l, int C, int lgC) {
+    if (lgC >= 0) {
+        const int sh = l * lgC;
+        return sh >= 63 ? 0 : (t >> sh);
+    }
+    for (int i = 0; i < l && t > 0; ++i) t /= C;
+    return t;
+}
+
+// The first scored level l* of a query at position t (0 if none): the highest
+// l >= 1 whose full list [0..a^(l)] has more than k entries.  Every level above it
+// selects its whole list, so A^(l*) = [0..a^(l*)].
+__device__ __forceinline__ int first_scored_level(int64_t t, int C, int lgC, int k) {
+    int lstar = 0, l = 0;
     int64_t p = t;
     while (p > 0 && l + 1 < kMaxLevels) {
-        p /= C;
+        p = cdiv64(p, C, lgC);
         ++l;
-        a[l] = p;
         if (p >= k) lstar = l;
     }
-    for (int r = l + 1; r < kMaxLevels; ++r) a[r] = 0;
     return lstar;
 }
 
 // |A^(level)| for a query whose first scored level is lstar >= level (Eq.3 sizes:
-// the list of l* is [0..a^(l*)], each lower list holds the C children of the
-// min(k, |A|) - 1 selected non-current nodes plus the current node's clamped
-// children).
-__device__ __forceinline__ int list_size(const int64_t* a, int lstar, int level, int C, int k) {
-    if (lstar == 0) return (int)(a[0] + 1);
-    int nA = (int)(a[lstar] + 1);
+// each list below l* holds the C children of the min(k, |A|) - 1 selected
+// non-current nodes plus the current node's children clamped at a^(l-1)).
+__device__ __forceinline__ int list_size(int64_t t, int lstar, int level, int C, int lgC, int k) {
+    if (lstar == 0) return (int)(t + 1);
+    int64_t al = apow(t, lstar, C, lgC);
+    int nA = (int)(al + 1);
     for (int l = lstar; l > level; --l) {
-        int nS = nA < k ? nA : k;
-        nA = C * (nS - 1) + (int)(a[l - 1] - (int64_t)C * a[l] + 1);
+        const int64_t alm1 = apow(t, l - 1, C, lgC);
+        const int nS = nA < k ? nA : k;
+        nA = C * (nS - 1) + (int)(alm1 - (int64_t)C * al + 1);
+        al = alm1;
     }
     return nA;
 }
@@ -214,6 +233,50 @@ struct ProfHook {
 inline void prof_mark(const ProfHook* p, int which, bool before, cudaStream_t s) {
     if (p == nullptr || p->which != which || p->start == nullptr) return;
     cudaEventRecordWithFlags(before ? p->start : p->stop, s, cudaEventRecordExternal);
+}
+
+// ----------------------------------------------------------------------------
+// TMA bulk copies into shared memory, completed on an mbarrier (no multicast)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+// One wait on a phase of an mbarrier: the thread is suspended in hardware until the
+// phase completes or about `hint_ns` nanoseconds pass (no issue slots are spent
+// spinning).  Returns whether the phase completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+// Bounded wait for a phase of an mbarrier: gives up after kWaitPolls suspended
+// waits of up to kWaitHintNs each (about one second in total), records
+// kStatusTimeout and returns false.  Never waits forever.
+constexpr uint32_t kWaitHintNs = 20000;
+constexpr uint32_t kWaitPolls = 50000;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    for (uint32_t i = 0; i < kWaitPolls; ++i)
+        if (mbar_try_wait(bar, parity, kWaitHintNs)) return true;
+    atomicCAS(status, 0u, 3u);
+    return false;
 }
 
 // ----------------------------------------------------------------------------

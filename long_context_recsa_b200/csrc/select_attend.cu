@@ -3,20 +3,29 @@
 // summaries of unselected candidates (Eq.4, "Unified Softmax"), sm_100a.
 //
 // Work unit: one (query, KV head).  For each level l >= 1 a cluster of SPL CTAs
-// splits the unit's candidate list A^(l) into contiguous chunks.  Each CTA
-//   1. rotates the G query heads to position p_q = |A|-1 and every candidate key
-//      of its chunk to its list index (cos/sin from an fp64-computed table),
-//      keeping the per-head logits in shared memory (never in global memory);
-//   2. picks its local top-(k-1) by (mean logit desc, index asc) with a radix
-//      select, exchanges the local lists through distributed shared memory, and
-//      every CTA selects the global top-(k-1) from the merged lists (the global
-//      winners are a subset of the local winners);
-//   3. writes S^(l) in ascending node order (rank = prefix count in list order;
-//      the current node is last), and accumulates the split-softmax partial
-//      (max, sum, weighted V) of its unselected candidates: the summaries.
-// Entry j of the next list is node C*S[j/C] + j%C (a "slot" r*C + c), so lists
-// are never materialised.  Level 0 runs the same scoring over A^(0) with every
-// entry included; a combine kernel merges all partials into the output.
+// splits the unit's candidate list A^(l) into contiguous chunks of whole parent
+// groups (C entries).  Each CTA
+//   1. scores its chunk: the G query heads are rotated once per parent group
+//      and every key by its child offset (slot-based rotation splitting, below);
+//      per-head logits stay in shared memory, never in global memory;
+//   2. exchanges the chunk's importance keys (mean logit, order-preserving
+//      uint32) with the other CTAs of the cluster through distributed shared
+//      memory, so that every CTA holds all |A|-1 keys in list order, and runs an
+//      exact radix select of the top k-1 (ties to the lower list position, which
+//      is the lower node index because lists are ascending);
+//   3. writes its part of S^(l) (rank = number of selected entries before it;
+//      the current node is last), prefetches the children of its selected nodes
+//      (the next level's rows) into L2, and accumulates the split-softmax partial
+//      (max, sum, weighted V) of its unselected entries: the summaries.
+// Entry j of the next list is node C*S[j/C] + j%C, so lists are never
+// materialised.  Level 0 scores A^(0) the same way with every entry included; the
+// last level-0 CTA of a unit merges all partials of the unit into the output.
+//
+// Slot-based rotation splitting: entry j = C*r + c sits at candidate-local
+// position j and the query at p_q = |A|-1, and
+//     <R(p_q) q, R(j) K> = <R(p_q - C r) q, R(c) K>,
+// so the query is rotated once per parent group r and each key only by one of C
+// fixed rotations R(0..C-1), staged in shared memory.
 #include <cooperative_groups.h>
 
 #include "recsa_internal.cuh"
@@ -38,33 +47,42 @@ struct Shape {
 // shared-memory layout of the select/attend kernels
 // ----------------------------------------------------------------------------
 struct Smem {
-    size_t qrot, s, key, rank, flag, ulist, par, lkey, lidx, mkey, midx, hist, red, misc, total;
+    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, samp, misc, bars, ring, red, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
-__host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int spl) {
+// CH: entries per CTA chunk; NA: largest list (C*k), 0 when no key exchange is
+// needed; ring_bytes: the warps' staging slots.  The reduction buffer reuses the
+// ring once every block has been consumed.
+__host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, int NA,
+                                            int ring_bytes) {
     Smem L;
-    const int K1 = k - 1 > 0 ? k - 1 : 1;
-    const int RN = CH > spl * K1 ? CH : spl * K1;
     size_t o = 0;
-    L.qrot = o;  o = align16(o + sizeof(float) * G * D);
+    L.qsm = o;   o = align16(o + sizeof(float) * G * D);
+    L.rc4 = o;   o = align16(o + sizeof(float2) * C * (D / 2));
     L.s = o;     o = align16(o + sizeof(float) * G * CH);
     L.key = o;   o = align16(o + sizeof(uint32_t) * CH);
-    L.rank = o;  o = align16(o + sizeof(int) * RN);
+    L.nodes = o; o = align16(o + sizeof(int) * CH);
     L.flag = o;  o = align16(o + sizeof(unsigned char) * CH);
-    L.ulist = o; o = align16(o + sizeof(int) * CH);
     L.par = o;   o = align16(o + sizeof(int) * k);
-    L.lkey = o;  o = align16(o + sizeof(uint32_t) * K1);
-    L.lidx = o;  o = align16(o + sizeof(int) * K1);
-    L.mkey = o;  o = align16(o + sizeof(uint32_t) * spl * K1);
-    L.midx = o;  o = align16(o + sizeof(int) * spl * K1);
-    L.hist = o;  o = align16(o + sizeof(uint32_t) * 256);
-    L.red = o;   o = align16(o + sizeof(float) * kWarps * G * D);
+    L.mkey = o;  o = align16(o + sizeof(uint32_t) * NA);
+    L.hist = o;  o = align16(o + sizeof(uint32_t) * 512);
+    L.samp = o;  o = align16(o + sizeof(uint32_t) * (NA > 0 ? kThreads : 0));
     L.misc = o;  o = align16(o + sizeof(int) * 64);
+    L.bars = o;  o = align16(o + sizeof(uint64_t) * kWarps * 2);
+    o = (o + 127) & ~size_t(127);
+    L.ring = o;
+    L.red = o;
+    const size_t red_bytes = sizeof(float) * kWarps * G * (D + 1);
+    o += (size_t)ring_bytes > red_bytes ? (size_t)ring_bytes : red_bytes;
     L.total = o;
     return L;
 }
+
+// misc slots
+enum { kMiscDigit = 0, kMiscAbove = 1, kMiscCount = 2, kMiscScan = 4 /* kWarps+1 */,
+       kMiscFloat = 16 /* 2*G floats */, kMiscLast = 40, kMiscN = 41 };
 
 // ----------------------------------------------------------------------------
 // block-wide primitives (kThreads threads)
@@ -81,14 +99,16 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int& total) 
     }
     if (lane == 31) scratch[warp] = x;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int tw = scratch[w];
-            scratch[w] = run;
-            run += tw;
+    if (threadIdx.x < 32) {
+        const int w = threadIdx.x < kWarps ? scratch[threadIdx.x] : 0;
+        int inc = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, inc, o);
+            if (threadIdx.x >= o) inc += y;
         }
-        scratch[kWarps] = run;
+        if (threadIdx.x < kWarps) scratch[threadIdx.x] = inc - w;
+        if (threadIdx.x == kWarps - 1) scratch[kWarps] = inc;
     }
     __syncthreads();
     const int off = scratch[warp] + x - v;
@@ -97,36 +117,41 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int& total) 
     return off;
 }
 
-// Exact top-K of n keys by (key desc, position asc).  rank[i] receives the rank of
-// item i among the selected items in position order, or -1.  MSB-first radix
-// select over 8-bit digits finds the threshold key T and how many items equal to T
-// are needed; those are the lowest-positioned ones.
-__device__ void block_topk_rank(const uint32_t* keys, int n, int K, int* rank, uint32_t* hist,
-                                int* misc) {
-    const int tid = threadIdx.x;
-    if (K >= n || K <= 0) {
-        for (int i = tid; i < n; i += kThreads) rank[i] = (K >= n) ? i : -1;
-        __syncthreads();
-        return;
-    }
+// Exact threshold of the top K of n keys (0 < K < n): T is the K-th largest key,
+// need_eq how many keys equal to T belong to the top K, cnt_eq how many keys equal
+// T.  MSB-first radix select over 8-bit digits; histogram updates are aggregated
+// per warp (__match_any_sync) because the leading digits of float keys fall into
+// a few bins.  hist: 512 words (two alternating 256-bin histograms).
+__device__ void block_threshold(const uint32_t* keys, int n, int K, uint32_t* hist, int* misc,
+                                uint32_t& T, int& need_eq, int& cnt_eq, int stride = 1) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int i = tid; i < 512; i += kThreads) hist[i] = 0u;
+    __syncthreads();
     uint32_t prefix = 0, mask = 0;
-    int rem = K;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += kThreads) hist[i] = 0u;
-        __syncthreads();
-        for (int i = tid; i < n; i += kThreads) {
-            const uint32_t kk = keys[i];
-            if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1u);
+    int rem = K, cnt = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        uint32_t* h = hist + (pass & 1) * 256;
+        uint32_t* hn = hist + ((pass + 1) & 1) * 256;
+        for (int i0 = 0; i0 < n; i0 += kThreads) {
+            const int i = i0 + tid;
+            const uint32_t kk = i < n ? keys[i * stride] : 0u;
+            const bool in = i < n && (kk & mask) == prefix;
+            const uint32_t dig = in ? ((kk >> shift) & 255u) : 256u;
+            const unsigned same = __match_any_sync(kFull, dig);
+            if (in && lane == __ffs(same) - 1) atomicAdd(&h[dig], (uint32_t)__popc(same));
         }
+        if (pass > 0)
+            for (int i = tid; i < 256; i += kThreads) hn[i] = 0u;   // last read by the previous scan
         __syncthreads();
         if (tid < 32) {
-            const int lane = tid;
-            uint32_t cnt[8];
+            uint32_t c8[8];
             uint32_t tot = 0;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                cnt[u] = hist[255 - 8 * lane - u];
-                tot += cnt[u];
+                c8[u] = h[255 - 8 * lane - u];
+                tot += c8[u];
             }
             uint32_t incl = tot;
 #pragma unroll
@@ -139,146 +164,369 @@ __device__ void block_topk_rank(const uint32_t* keys, int n, int K, int* rank, u
                 uint32_t run = excl;
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    if (run + cnt[u] >= (uint32_t)rem) {
-                        misc[0] = 255 - 8 * lane - u;
-                        misc[1] = (int)run;
+                    if (run + c8[u] >= (uint32_t)rem) {
+                        misc[kMiscDigit] = 255 - 8 * lane - u;
+                        misc[kMiscAbove] = (int)run;
+                        misc[kMiscCount] = (int)c8[u];
                         break;
                     }
-                    run += cnt[u];
+                    run += c8[u];
                 }
             }
         }
         __syncthreads();
-        const int digit = misc[0], above = misc[1];
-        rem -= above;
+        const int digit = misc[kMiscDigit];
+        rem -= misc[kMiscAbove];
+        cnt = misc[kMiscCount];
         prefix |= (uint32_t)digit << shift;
         mask |= 255u << shift;
-        __syncthreads();
-    }
-    const uint32_t T = prefix;
-    const int need_eq = rem;
-    // ties: the first need_eq items equal to T (position order)
-    const int ipt = (n + kThreads - 1) / kThreads;
-    const int i0 = tid * ipt, i1 = min(n, i0 + ipt);
-    int ceq = 0;
-    for (int i = i0; i < i1; ++i) ceq += (keys[i] == T);
-    int tot;
-    int eq_rank = block_excl_scan(ceq, misc + 2, tot);
-    int csel = 0;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t kk = keys[i];
-        bool sel = kk > T;
-        if (kk == T) { sel = eq_rank < need_eq; ++eq_rank; }
-        rank[i] = sel ? 1 : 0;
-        csel += sel;
-    }
-    int r = block_excl_scan(csel, misc + 2, tot);
-    for (int i = i0; i < i1; ++i) {
-        if (rank[i]) rank[i] = r++;
-        else rank[i] = -1;
     }
     __syncthreads();
+    T = prefix;
+    need_eq = rem;
+    cnt_eq = cnt;
+}
+
+// Selection ranks of n keys in list order given the threshold: selected = key > T,
+// or key == T among the first need_eq such keys.  Calls fn(i, rank) for every
+// selected item i in [lo, hi).  Returns the number of selected items.
+template <typename Fn>
+__device__ int block_select_ranks(const uint32_t* keys, int n, uint32_t T, int need_eq, int cnt_eq,
+                                  int lo, int hi, int* misc, Fn fn, int stride = 1) {
+    const int ipt = (n + kThreads - 1) / kThreads;
+    const int i0 = threadIdx.x * ipt, i1 = min(n, i0 + ipt);
+    const bool all_eq = (cnt_eq == need_eq);
+    int eq_rank = 0, tot;
+    if (!all_eq) {
+        int ceq = 0;
+        for (int i = i0; i < i1; ++i) ceq += (keys[i * stride] == T);
+        eq_rank = block_excl_scan(ceq, misc + kMiscScan, tot);
+    }
+    int csel = 0;
+    {
+        int er = eq_rank;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t kk = keys[i * stride];
+            bool sel = kk > T;
+            if (kk == T) { sel = all_eq || er < need_eq; ++er; }
+            csel += sel;
+        }
+    }
+    int r = block_excl_scan(csel, misc + kMiscScan, tot);
+    {
+        int er = eq_rank;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t kk = keys[i * stride];
+            bool sel = kk > T;
+            if (kk == T) { sel = all_eq || er < need_eq; ++er; }
+            if (sel) {
+                if (i >= lo && i < hi) fn(i, r);
+                ++r;
+            }
+        }
+    }
+    return tot;
+}
+
+// Exact top-K (0 < K < M) of the M keys of mkey in list order; calls mark(j, rank)
+// for every selected list position j in [lo, hi), rank = its position among the
+// selected in list order.  A threshold T0 estimated from a 256-key sample bounds a
+// compact candidate list (keys >= T0, in list order, packed as (key, position) in
+// mkey); the exact radix select and the ranks then run on that list.  When the
+// estimate misses (fewer than K or more than kCap candidates) the whole list is
+// used.  Both paths give the same result.
+template <typename Fn>
+__device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, uint32_t* sample, int* misc,
+                            int lo, int hi, Fn mark) {
+    constexpr int NS = kThreads;     // sample size, one key per thread
+    constexpr int IPT = 16;          // keys per thread held in registers while compacting
+    constexpr int kCap = 2048;       // compact list capacity ((key, position) pairs in mkey)
+    const int tid = threadIdx.x;
+    uint32_t T;
+    int need_eq, cnt_eq, n0 = 0;
+    bool compact = false;
+    if (M > 2 * NS && M <= IPT * kThreads) {
+        sample[tid] = mkey[(int)(((int64_t)tid * M) / NS)];
+        __syncthreads();
+        int q = (int)(((int64_t)(K + (3 * K) / 5 + 32) * NS + M - 1) / M);
+        q = min(max(q, 1), NS - 1);
+        uint32_t T0;
+        int ne0, ce0;
+        block_threshold(sample, NS, q, hist, misc, T0, ne0, ce0);
+        const int i0 = tid * IPT;
+        uint32_t kr[IPT];
+        int c = 0;
+#pragma unroll
+        for (int u = 0; u < IPT; ++u) {
+            const int i = i0 + u;
+            kr[u] = i < M ? mkey[i] : 0u;
+            c += (i < M && kr[u] >= T0) ? 1 : 0;
+        }
+        int tot;
+        int off = block_excl_scan(c, misc + kMiscScan, tot);   // every load is done past its barriers
+        if (tot >= K && tot <= kCap) {
+            uint2* pairs = reinterpret_cast<uint2*>(mkey);
+#pragma unroll
+            for (int u = 0; u < IPT; ++u) {
+                const int i = i0 + u;
+                if (i < M && kr[u] >= T0) pairs[off++] = make_uint2(kr[u], (uint32_t)i);
+            }
+            __syncthreads();
+            compact = true;
+            n0 = tot;
+        }
+    }
+    if (compact) {
+        const uint2* pairs = reinterpret_cast<const uint2*>(mkey);
+        block_threshold(mkey, n0, K, hist, misc, T, need_eq, cnt_eq, 2);
+        block_select_ranks(
+            mkey, n0, T, need_eq, cnt_eq, 0, n0, misc,
+            [&](int ic, int r) {
+                const int j = (int)pairs[ic].y;
+                if (j >= lo && j < hi) mark(j, r);
+            },
+            2);
+    } else {
+        block_threshold(mkey, M, K, hist, misc, T, need_eq, cnt_eq);
+        block_select_ranks(mkey, M, T, need_eq, cnt_eq, lo, hi, misc, mark);
+    }
 }
 
 // ----------------------------------------------------------------------------
-// scoring: s[g][r] = scale * <R(p_q) q_g, R(j) K_node(j)>, j = j0 + r
+// L2 prefetch: a bulk asynchronous request that holds no registers or shared
+// memory; the rows are in L2 when the loads reach them.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// cnt consecutive rows starting at row `first` (row stride rs), K and V.
+template <typename T, int D>
+__device__ __forceinline__ void prefetch_children(const T* kb, const T* vb, int64_t rs,
+                                                  int64_t first, int cnt) {
+    constexpr uint32_t kRow = D * sizeof(T);
+    if (rs == D) {
+        prefetch_l2(kb + first * D, cnt * kRow);
+        prefetch_l2(vb + first * D, cnt * kRow);
+    } else {
+        for (int c = 0; c < cnt; ++c) {
+            prefetch_l2(kb + (first + c) * rs, kRow);
+            prefetch_l2(vb + (first + c) * rs, kRow);
+        }
+    }
+}
+
+// 16 loaded bytes as VEC/2 fp32 pairs (elements 2i, 2i+1).
+template <typename T>
+__device__ __forceinline__ void unpack_pairs(const uint4& w, float2* out);
+template <>
+__device__ __forceinline__ void unpack_pairs<float>(const uint4& w, float2* out) {
+    out[0] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+    out[1] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+}
+template <>
+__device__ __forceinline__ void unpack_pairs<__nv_bfloat16>(const uint4& w, float2* out) {
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        out[i] = make_float2(__uint_as_float(x[i] << 16), __uint_as_float(x[i] & 0xffff0000u));
+}
+
+// Reduce-scatter of N register values over the KG lanes (a power of two) of a
+// key group: afterwards v[0 .. N/KG) of lane c8 hold the group sums of original
+// indices [c8*N/KG, (c8+1)*N/KG).  Each stage halves the live values: lanes whose
+// stage bit is set keep the upper half and send the lower one.
+template <int N, int KG>
+__device__ __forceinline__ void reduce_scatter(float (&v)[N], int c8) {
+#pragma unroll
+    for (int o = KG / 2, n = N; o >= 1; o >>= 1, n >>= 1) {
+        const bool up = (c8 & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float lo = v[i], hi = v[i + n / 2];
+            const float send = up ? lo : hi;
+            const float keep = up ? hi : lo;
+            v[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Per-warp ring of parent-group blocks (C rows of K or V) staged in shared memory
+// by TMA bulk copies.  Block q of a warp goes to slot q % nsw; a slot is re-armed
+// only after the warp has consumed its previous block, so each warp keeps nsw
+// blocks in flight without holding registers.
+// ----------------------------------------------------------------------------
+struct WarpRing {
+    unsigned char* slots;
+    uint64_t* bars;
+    int nsw, slot_bytes;
+    uint32_t* status;
+};
+
+// Issue block q: rows [first, first + cnt) of a table with row stride rs.  One lane.
+template <typename T, int D>
+__device__ __forceinline__ void ring_issue(const WarpRing& R, int q, const T* base, int64_t rs,
+                                           int64_t first, int cnt) {
+    constexpr uint32_t kRow = D * sizeof(T);
+    const int s = q % R.nsw;
+    unsigned char* dst = R.slots + (size_t)s * R.slot_bytes;
+    mbar_expect_tx(&R.bars[s], (uint32_t)cnt * kRow);
+    if (rs == D) {
+        bulk_g2s(dst, base + first * D, (uint32_t)cnt * kRow, &R.bars[s]);
+    } else {
+        for (int r = 0; r < cnt; ++r) bulk_g2s(dst + r * kRow, base + (first + r) * rs, kRow, &R.bars[s]);
+    }
+}
+
+// Wait (bounded) for block q; all lanes of the warp.
+__device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int q) {
+    const int s = q % R.nsw;
+    mbar_wait_bounded(&R.bars[s], (uint32_t)((q / R.nsw) & 1), R.status);
+    return R.slots + (size_t)s * R.slot_bytes;
+}
+
+// ----------------------------------------------------------------------------
+// Scores of one parent group staged in shared memory: row c of blk is the key of
+// list entry jb + c (c < nch).  s[g][r] = scale * <R(p_q - jb) q_g, R(c) K>, the
+// order-preserving key of the mean over heads, and the node index first + c,
+// at r = jb - j0 + c.  Packed fp32x2 arithmetic; each key is reduced over its
+// KG lanes by a reduce-scatter.
 // ----------------------------------------------------------------------------
 template <typename T, int D, int G, bool WITH_KEY>
-__device__ __forceinline__ void score_chunk(const T* kbase, int64_t rs, const float2* rope, int j0,
-                                            int n, bool identity, const int* par, int C,
-                                            float scale, const float* qrot, float* s,
-                                            uint32_t* key, int CH) {
+__device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, int j0, int nch,
+                                             int64_t first, const float2* rope, int p_q,
+                                             const float4* rc4, const float* qsm, float scale,
+                                             float* s, uint32_t* key, int* nodes, int CH) {
     using S = Shape<T, D>;
-    constexpr int VEC = S::VEC;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int c = lane % S::KG, kg = lane / S::KG;
-    float qlo[G][VEC], qhi[G][VEC];
+    constexpr int VEC = S::VEC, KG = S::KG, KPW = S::KPW, H = D / 2, V2 = VEC / 2;
+    constexpr int kRow = D * (int)sizeof(T);
+    constexpr int U = 4;                       // keys per lane per batch
+    constexpr int NV = U * G;                  // values reduced over a key group
+    constexpr int R = NV / KG;                 // values per lane after reduce-scatter
+    constexpr bool RS = (NV % KG == 0) && (R >= 1) && (G % (R > 0 ? R : 1) == 0);
+    const int lane = threadIdx.x & 31;
+    const int c8 = lane % KG, kg = lane / KG;
+    float2 qlo[G][V2], qhi[G][V2];
+    {
+        const float4* qcs =
+            reinterpret_cast<const float4*>(rope + (int64_t)(p_q - jb) * H + c8 * VEC);
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int w = 0; w < V2; ++w) {
+            const float4 cs = __ldg(qcs + w);   // (cos v, sin v, cos v+1, sin v+1)
+            const float2 co = make_float2(cs.x, cs.z);
+            const float2 si = make_float2(cs.y, cs.w);
+            const float2 ns = make_float2(-cs.y, -cs.w);
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-            qlo[g][v] = qrot[g * D + c * VEC + v];
-            qhi[g][v] = qrot[g * D + D / 2 + c * VEC + v];
+            for (int g = 0; g < G; ++g) {
+                const float2 x1 = *reinterpret_cast<const float2*>(qsm + g * D + c8 * VEC + 2 * w);
+                const float2 x2 = *reinterpret_cast<const float2*>(qsm + g * D + H + c8 * VEC + 2 * w);
+                qlo[g][w] = __ffma2_rn(x2, ns, __fmul2_rn(x1, co));
+                qhi[g][w] = __ffma2_rn(x1, si, __fmul2_rn(x2, co));
+            }
         }
-    for (int base = warp * S::KPW; base < n; base += kWarps * S::KPW) {
-        const int r = base + kg;
-        const bool act = r < n;
-        float acc[G];
+    }
+    for (int cb = 0; cb < nch; cb += KPW * U) {
+        float v[NV];
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = 0.f;
-        if (act) {
-            const int j = j0 + r;
-            const int64_t node = identity ? (int64_t)j : (int64_t)C * par[j / C] + (j % C);
-            const T* row = kbase + node * rs;
-            float klo[VEC], khi[VEC];
-            load16_nc<T>(row + c * VEC, klo);
-            load16_nc<T>(row + D / 2 + c * VEC, khi);
-            const float4* cs4 = reinterpret_cast<const float4*>(rope + (int64_t)j * (D / 2) + c * VEC);
+        for (int u = 0; u < U; ++u) {
+            const int c = cb + u * KPW + kg;
+            float2 a2[G];
 #pragma unroll
-            for (int v2 = 0; v2 < VEC / 2; ++v2) {
-                const float4 cs = __ldg(cs4 + v2);
+            for (int g = 0; g < G; ++g) a2[g] = make_float2(0.f, 0.f);
+            if (c < nch) {
+                const unsigned char* row = blk + c * kRow;
+                float2 kl[V2], kh[V2];
+                unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + c8 * 16), kl);
+                unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + H * (int)sizeof(T) + c8 * 16), kh);
+                const float4* rc = rc4 + (c * H + c8 * VEC) / 2;
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int v = 2 * v2 + u;
-                    const float co = u ? cs.z : cs.x, si = u ? cs.w : cs.y;
-                    const float a = klo[v] * co - khi[v] * si;
-                    const float bb = klo[v] * si + khi[v] * co;
+                for (int w = 0; w < V2; ++w) {
+                    const float4 cs = rc[w];   // (cos v, cos v+1, sin v, sin v+1) of c * theta
+                    const float2 co = make_float2(cs.x, cs.y);
+                    const float2 si = make_float2(cs.z, cs.w);
+                    const float2 ns = __fmul2_rn(si, make_float2(-1.f, -1.f));
+                    const float2 ka = __ffma2_rn(kh[w], ns, __fmul2_rn(kl[w], co));
+                    const float2 kb = __ffma2_rn(kl[w], si, __fmul2_rn(kh[w], co));
 #pragma unroll
-                    for (int g = 0; g < G; ++g) acc[g] += qlo[g][v] * a + qhi[g][v] * bb;
+                    for (int g = 0; g < G; ++g) {
+                        a2[g] = __ffma2_rn(qlo[g][w], ka, a2[g]);
+                        a2[g] = __ffma2_rn(qhi[g][w], kb, a2[g]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) v[u * G + g] = a2[g].x + a2[g].y;
+        }
+        if constexpr (RS) {
+            reduce_scatter<NV, KG>(v, c8);
+            const int u = (c8 * R) / G, g0 = (c8 * R) % G;
+            const int c = cb + u * KPW + kg;
+            float imp = 0.f;
+#pragma unroll
+            for (int i = 0; i < R; ++i) imp += v[i];
+#pragma unroll
+            for (int o = 1; o < G / R; o <<= 1) imp += __shfl_xor_sync(kFull, imp, o);
+            if (c < nch) {
+                const int r = jb - j0 + c;
+#pragma unroll
+                for (int i = 0; i < R; ++i) s[(g0 + i) * CH + r] = v[i] * scale;
+                if (g0 == 0) {
+                    nodes[r] = (int)(first + c);
+                    if (WITH_KEY) key[r] = ordered_key(imp * scale * (1.0f / G));
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < NV; ++i)
+#pragma unroll
+                for (int o = 1; o < KG; o <<= 1) v[i] += __shfl_xor_sync(kFull, v[i], o);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = cb + u * KPW + kg;
+                if (c < nch && c8 == 0) {
+                    const int r = jb - j0 + c;
+                    float imp = 0.f;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        s[g * CH + r] = v[u * G + g] * scale;
+                        imp += v[u * G + g];
+                    }
+                    nodes[r] = (int)(first + c);
+                    if (WITH_KEY) key[r] = ordered_key(imp * scale * (1.0f / G));
                 }
             }
         }
-#pragma unroll
-        for (int o = 1; o < S::KG; o <<= 1)
-#pragma unroll
-            for (int g = 0; g < G; ++g) acc[g] += __shfl_xor_sync(kFull, acc[g], o);
-        if (act && c == 0) {
-            float imp = 0.f;
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float sv = acc[g] * scale;
-                s[g * CH + r] = sv;
-                imp += sv;
-            }
-            if (WITH_KEY) key[r] = ordered_key(imp * (1.0f / G));
-        }
     }
 }
 
-// Rotate the G query heads of KV head kvh to position p_q into qrot[G][D].
+// Unrotated query heads of one KV head (fp32) and the C child rotations R(c)
+// (cos, sin, -sin) into shared memory.
 template <typename T, int D, int G>
-__device__ __forceinline__ void rotate_query(const T* qrow /* head kvh*G */, const float2* rope,
-                                             int p_q, float* qrot) {
-    for (int i = threadIdx.x; i < G * (D / 2); i += kThreads) {
-        const int g = i / (D / 2), pr = i % (D / 2);
-        const float x1 = (float)qrow[g * D + pr];
-        const float x2 = (float)qrow[g * D + pr + D / 2];
-        const float2 cs = rope[(int64_t)p_q * (D / 2) + pr];
-        qrot[g * D + pr] = x1 * cs.x - x2 * cs.y;
-        qrot[g * D + pr + D / 2] = x1 * cs.y + x2 * cs.x;
+__device__ __forceinline__ void stage_query(const T* qrow, const float2* rope, int C, float* qsm,
+                                            float4* rc4) {
+    for (int i = threadIdx.x; i < G * D; i += kThreads) qsm[i] = (float)qrow[i];
+    // R(c), c < C, as (cos v, cos v+1, sin v, sin v+1) for pair couples (v, v+1)
+    for (int i = threadIdx.x; i < C * (D / 4); i += kThreads) {
+        const float2 a = rope[2 * i], bb = rope[2 * i + 1];
+        rc4[i] = make_float4(a.x, bb.x, a.y, bb.y);
     }
 }
 
-// Softmax partial over the chunk entries listed in ulist (chunk-relative indices):
-// m_g = max s, p = exp(s - m) (in place), l_g = sum p, o_g = sum p V.  Writes the
-// partial record [G][D+2] = (o, m, l).  Empty list -> (0, -inf, 0).
-template <typename T, int D, int G>
-__device__ void softmax_partial(const T* vbase, int64_t rs, int j0, const int* ulist, int nu,
-                                bool identity, const int* par, int C, float* s, int CH,
-                                float* red, int* misc, float* outp) {
-    using S = Shape<T, D>;
-    constexpr int VEC = S::VEC;
+// Softmax weights of the included chunk entries (entry i < n with flag[i] == 0,
+// or every entry when flag is null): m_g = max s, s <- exp(s - m) in place, and
+// this thread's part of l_g = sum exp.  fm[0..G) receives m.
+template <int G>
+__device__ __forceinline__ void softmax_weights(float* s, int n, const unsigned char* flag, int CH,
+                                                float* red, float* fm, float* lsum) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float* fmisc = reinterpret_cast<float*>(misc);
-    // per-head max
     float mx[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
-    for (int u = threadIdx.x; u < nu; u += kThreads) {
-        const int r = ulist[u];
+    for (int i = threadIdx.x; i < n; i += kThreads)
+        if (!flag || flag[i] == 0)
 #pragma unroll
-        for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], s[g * CH + r]);
-    }
+            for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], s[g * CH + i]);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -289,86 +537,100 @@ __device__ void softmax_partial(const T* vbase, int64_t rs, int j0, const int* u
     if (threadIdx.x < G) {
         float m = -INFINITY;
         for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w * G + threadIdx.x]);
-        fmisc[threadIdx.x] = m;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int g = 0; g < G; ++g) mx[g] = fmisc[g];
-    // p = exp(s - m), per-head sums
-    float sm[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) sm[g] = 0.f;
-    for (int u = threadIdx.x; u < nu; u += kThreads) {
-        const int r = ulist[u];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float p = __expf(s[g * CH + r] - mx[g]);
-            s[g * CH + r] = p;
-            sm[g] += p;
-        }
+        fm[threadIdx.x] = m;
     }
     __syncthreads();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sm[g] += __shfl_xor_sync(kFull, sm[g], o);
-        if (lane == 0) red[warp * G + g] = sm[g];
+        mx[g] = fm[g];
+        lsum[g] = 0.f;
     }
-    __syncthreads();
-    if (threadIdx.x < G) {
-        float l = 0.f;
-        for (int w = 0; w < kWarps; ++w) l += red[w * G + threadIdx.x];
-        fmisc[G + threadIdx.x] = l;
-    }
-    __syncthreads();
-    // o = sum p V
-    const int c = lane % S::RPL, rr = lane / S::RPL;
-    float acc[G][VEC];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[g][e] = 0.f;
-#pragma unroll 4
-    for (int base = warp * S::RPW; base < nu; base += kWarps * S::RPW) {
-        const int u = base + rr;
-        if (u < nu) {
-            const int r = ulist[u];
-            const int j = j0 + r;
-            const int64_t node = identity ? (int64_t)j : (int64_t)C * par[j / C] + (j % C);
-            float v[VEC];
-            load16_nc<T>(vbase + node * rs + c * VEC, v);
+    for (int i = threadIdx.x; i < n; i += kThreads)
+        if (!flag || flag[i] == 0)
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float p = s[g * CH + r];
+                const float p = __expf(s[g * CH + i] - mx[g]);
+                s[g * CH + i] = p;
+                lsum[g] += p;
+            }
+    __syncthreads();
+}
+
+// o_g += p_g * V for the rows of one staged parent group: row c of blk is the
+// value of entry jb + c (c < nrow), skipped when flagged (selected).
+template <typename T, int D, int G>
+__device__ __forceinline__ void accum_parent(const unsigned char* blk, int jb, int j0, int nrow,
+                                             const unsigned char* flag, const float* s, int CH,
+                                             float2 (&acc)[G][VecOf<T>::N / 2]) {
+    using S = Shape<T, D>;
+    constexpr int V2 = S::VEC / 2;
+    constexpr int kRow = D * (int)sizeof(T);
+    const int lane = threadIdx.x & 31;
+    const int c = lane % S::RPL, rr = lane / S::RPL;
+#pragma unroll 4
+    for (int cb = 0; cb < nrow; cb += S::RPW) {
+        const int cr = cb + rr;
+        if (cr < nrow) {
+            const int r = jb - j0 + cr;
+            if (!flag || flag[r] == 0) {
+                float2 v[V2];
+                unpack_pairs<T>(*reinterpret_cast<const uint4*>(blk + cr * kRow + c * 16), v);
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[g][e] += p * v[e];
+                for (int g = 0; g < G; ++g) {
+                    const float p = s[g * CH + r];
+                    const float2 p2 = make_float2(p, p);
+#pragma unroll
+                    for (int e = 0; e < V2; ++e) acc[g][e] = __ffma2_rn(p2, v[e], acc[g][e]);
+                }
             }
         }
     }
+}
+
+// Cross-lane and cross-warp reduction of the value accumulators and l partials
+// into the partial record [G][D+2] = (o, m, l).  red must be free.
+template <typename T, int D, int G>
+__device__ __forceinline__ void finish_partial(float2 (&acc)[G][VecOf<T>::N / 2], float* lsum,
+                                               const float* fm, float* red, float* outp) {
+    using S = Shape<T, D>;
+    constexpr int VEC = S::VEC, V2 = VEC / 2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c = lane % S::RPL, rr = lane / S::RPL;
 #pragma unroll
     for (int o = S::RPL; o < 32; o <<= 1)
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[g][e] += __shfl_xor_sync(kFull, acc[g][e], o);
-    __syncthreads();   // red reused
+            for (int e = 0; e < V2; ++e) {
+                acc[g][e].x += __shfl_xor_sync(kFull, acc[g][e].x, o);
+                acc[g][e].y += __shfl_xor_sync(kFull, acc[g][e].y, o);
+            }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lsum[g] += __shfl_xor_sync(kFull, lsum[g], o);
     if (rr == 0) {
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) red[(warp * G + g) * D + c * VEC + e] = acc[g][e];
+            for (int e = 0; e < V2; ++e) {
+                red[(warp * G + g) * (D + 1) + c * VEC + 2 * e] = acc[g][e].x;
+                red[(warp * G + g) * (D + 1) + c * VEC + 2 * e + 1] = acc[g][e].y;
+            }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) red[(warp * G + g) * (D + 1) + D] = lsum[g];
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < G * D; i += kThreads) {
+    for (int i = threadIdx.x; i < G * (D + 1); i += kThreads) {
         float sum = 0.f;
-        for (int w = 0; w < kWarps; ++w) sum += red[w * G * D + i];
-        const int g = i / D, d = i % D;
-        outp[g * (D + 2) + d] = sum;
+        for (int w = 0; w < kWarps; ++w) sum += red[w * G * (D + 1) + i];
+        const int g = i / (D + 1), d = i % (D + 1);
+        if (d < D) outp[g * (D + 2) + d] = sum;
+        else outp[g * (D + 2) + D + 1] = sum;
     }
-    if (threadIdx.x < G) {
-        outp[threadIdx.x * (D + 2) + D] = fmisc[threadIdx.x];
-        outp[threadIdx.x * (D + 2) + D + 1] = fmisc[G + threadIdx.x];
-    }
+    if (threadIdx.x < G) outp[threadIdx.x * (D + 2) + D] = fm[threadIdx.x];
 }
 
 __device__ __forceinline__ void write_empty_partial(float* outp, int G, int D) {
@@ -378,52 +640,121 @@ __device__ __forceinline__ void write_empty_partial(float* outp, int G, int D) {
     }
 }
 
+// Log-sum-exp merge of a unit's partials into its G output heads.  Partials of
+// other CTAs are read through L2 (ld.global.cg).
+template <typename T, int D, int G>
+__device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL, T* out,
+                             float* wsh /* >= G*(NL*SPL+NS0) */, float* Lsh /* G */) {
+    const int nls = lstar * SPL;
+    const int ns = nls + NS0;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int g = warp; g < G; g += kWarps) {
+        float M = -INFINITY;
+        for (int i = lane; i < ns; i += 32) {
+            const int slot = i < nls ? i : NL * SPL + (i - nls);
+            M = fmaxf(M, __ldcg(P + (slot * G + g) * (D + 2) + D));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+        float L = 0.f;
+        for (int i = lane; i < ns; i += 32) {
+            const int slot = i < nls ? i : NL * SPL + (i - nls);
+            const float m = __ldcg(P + (slot * G + g) * (D + 2) + D);
+            const float l = __ldcg(P + (slot * G + g) * (D + 2) + D + 1);
+            const float w = l > 0.f ? __expf(m - M) : 0.f;
+            wsh[g * ns + i] = w;
+            L += w * l;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
+        if (lane == 0) Lsh[g] = L;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < G * D; e += kThreads) {
+        const int g = e / D, d = e % D;
+        float O = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < ns; ++i) {
+            const int slot = i < nls ? i : NL * SPL + (i - nls);
+            O += wsh[g * ns + i] * __ldcg(P + (slot * G + g) * (D + 2) + d);
+        }
+        const float L = Lsh[g];
+        out[e] = store_round_f<T>(L > 0.f ? O / L : 0.f);
+    }
+}
+
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------------
 // level l >= 1: score + RoPE + TopK + summaries (cluster of SPL CTAs per unit)
-// level 0 (L0 = true): score + softmax partial over A^(0) (NS0 CTAs per unit)
+// level 0 (L0 = true): score + softmax partial over A^(0) (NS0 CTAs per unit);
+// the last of them merges every partial of the unit into the output.
+// Each warp takes every kWarps-th parent group of the chunk; its K blocks and
+// then its V blocks stream through its ring, so V loads overlap the selection.
 // ----------------------------------------------------------------------------
 template <typename T, int D, int G, bool L0>
-__global__ void __launch_bounds__(kThreads) level_kernel(TreeView tv, WorkView wv, QueryView qv,
-                                                         int level, int CH) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int k = tv.k, C = tv.C;
-    const int K1 = k - 1;
+__global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkView wv, QueryView qv,
+                                                            int level, int CH, int NA, int nsw) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    constexpr int kRow = D * (int)sizeof(T);
+    constexpr int V2 = VecOf<T>::N / 2;
+    const int k = tv.k, C = tv.C, lgC = tv.lgC, K1 = k - 1, NL = wv.NL;
     const int nsplit = L0 ? wv.NS0 : wv.SPL;
-    const Smem SL = smem_layout(G, D, CH, k, L0 ? 1 : wv.SPL);
-    float* qrot = reinterpret_cast<float*>(smem + SL.qrot);
+    const int slot_bytes = C * kRow;
+    const Smem SL = smem_layout(G, D, CH, k, C, L0 ? 0 : NA, kWarps * nsw * slot_bytes);
+    float* qsm = reinterpret_cast<float*>(smem + SL.qsm);
+    float4* rc4 = reinterpret_cast<float4*>(smem + SL.rc4);
+
     float* s = reinterpret_cast<float*>(smem + SL.s);
     uint32_t* key = reinterpret_cast<uint32_t*>(smem + SL.key);
-    int* rank = reinterpret_cast<int*>(smem + SL.rank);
+    int* nodes = reinterpret_cast<int*>(smem + SL.nodes);
     unsigned char* flag = smem + SL.flag;
-    int* ulist = reinterpret_cast<int*>(smem + SL.ulist);
     int* par = reinterpret_cast<int*>(smem + SL.par);
-    uint32_t* lkey = reinterpret_cast<uint32_t*>(smem + SL.lkey);
-    int* lidx = reinterpret_cast<int*>(smem + SL.lidx);
     uint32_t* mkey = reinterpret_cast<uint32_t*>(smem + SL.mkey);
-    int* midx = reinterpret_cast<int*>(smem + SL.midx);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + SL.hist);
-    float* red = reinterpret_cast<float*>(smem + SL.red);
+    uint32_t* samp = reinterpret_cast<uint32_t*>(smem + SL.samp);
     int* misc = reinterpret_cast<int*>(smem + SL.misc);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bars);
+    unsigned char* ring = smem + SL.ring;
+    float* red = reinterpret_cast<float*>(smem + SL.red);   // reuses the ring after the last block
+    float* fm = reinterpret_cast<float*>(misc + kMiscFloat);
 
     const int unit = blockIdx.y;
     const int split = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qloc = unit / tv.Hkv, kvh = unit % tv.Hkv;
-    int b, gq;
-    int64_t t;
-    const bool valid = query_pos(qv, wv, qloc, b, t, gq);
-    int64_t a[kMaxLevels];
-    const int lstar = valid ? first_scored_level(t, C, k, a) : 0;
-    const int NL = wv.NL;
+    const int gq = qv.q_begin + qloc;
+    const int b = gq / qv.n_per_b;
+    const int64_t len = wv.lens[b];
+    // loads that depend only on the unit are issued together: query heads, child
+    // rotations, and the parent list S^(level+1) when there is one
+    const T* qrow = reinterpret_cast<const T*>(qv.q) + ((int64_t)gq * tv.Hq + kvh * G) * D;
+    stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
+    if (L0 ? NL >= 1 : level < NL) {
+        const int32_t* src = wv.sel + ((int64_t)unit * NL + level) * k;
+        for (int i = threadIdx.x; i < k; i += kThreads) par[i] = src[i];
+    }
+    if (threadIdx.x < kWarps * nsw) mbar_init(&bars[threadIdx.x], 1);
+    mbar_fence_init();
+    const int64_t t = (qv.mode == 0) ? len - 1 : qv.pos0 + (gq - b * qv.n_per_b);
+    const bool valid = t >= 0 && t < len;
+    const int lstar = valid ? first_scored_level(t, C, lgC, k) : 0;
     int32_t* cnt_ws = wv.cnt + (int64_t)unit * (NL + 1);
     int32_t* cnt_usr = qv.cnt_out ? qv.cnt_out + ((int64_t)gq * tv.Hkv + kvh) * (NL + 1) : nullptr;
     float* part = wv.part + (int64_t)unit * wv.NSLOT * G * (D + 2);
+    __syncthreads();
 
     if (!L0 && (!valid || level > lstar)) {
-        // level not scored for this query: all of its list is selected
+        // not scored for this query: its whole list is selected
         if (split == 0) {
-            for (int i = threadIdx.x; i < k; i += kThreads) {
-                if (qv.sel_out) qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k + i] = -1;
-            }
+            if (qv.sel_out)
+                for (int i = threadIdx.x; i < k; i += kThreads)
+                    qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k + i] = -1;
             if (threadIdx.x == 0) {
                 cnt_ws[level] = 0;
                 if (cnt_usr) cnt_usr[level] = 0;
@@ -432,24 +763,25 @@ __global__ void __launch_bounds__(kThreads) level_kernel(TreeView tv, WorkView w
         return;
     }
     if (L0 && !valid) {
-        if (split == 0 && threadIdx.x == 0) {
-            cnt_ws[0] = 0;
-            if (cnt_usr) cnt_usr[0] = 0;
+        // nothing to attend (empty sequence, or a prefill row beyond the length)
+        if (split == 0) {
+            T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
+            for (int i = threadIdx.x; i < G * D; i += kThreads) out[i] = store_round_f<T>(0.f);
+            if (threadIdx.x == 0) {
+                cnt_ws[0] = 0;
+                if (cnt_usr) cnt_usr[0] = 0;
+                if (qv.mode == 1) set_status(wv.status, kStatusBadQuery);
+            }
         }
         return;
     }
 
-    const int nA = list_size(a, lstar, level, C, k);
+    const int nA = list_size(t, lstar, level, C, lgC, k);
     const bool identity = (level == lstar) || (L0 && lstar == 0);
-    if (!identity) {
-        const int32_t* src = wv.sel + ((int64_t)unit * NL + level) * k;   // S^(level+1)
-        for (int i = threadIdx.x; i < k; i += kThreads) par[i] = src[i];
-    }
-    const int p_q = nA - 1;
-    const T* qrow = reinterpret_cast<const T*>(qv.q) + ((int64_t)gq * tv.Hq + kvh * G) * D;
-    rotate_query<T, D, G>(qrow, wv.rope, p_q, qrot);
-    __syncthreads();
-
+    const int npar_all = cdiv(nA + C - 1, C, lgC);
+    const int chunk = ((npar_all + nsplit - 1) / nsplit) * C;
+    const int j0 = split * chunk;
+    const int j1 = min(nA, j0 + chunk);
     const T *kbase, *vbase;
     int64_t rs;
     if (L0) {
@@ -461,41 +793,25 @@ __global__ void __launch_bounds__(kThreads) level_kernel(TreeView tv, WorkView w
         vbase = level_v<T>(tv, level, b, kvh);
         rs = D;
     }
-    const int chunk = (nA + nsplit - 1) / nsplit;
-    const int j0 = split * chunk;
-    const int j1 = min(nA, j0 + chunk);
-
-    if (L0) {
-        const int n = max(0, j1 - j0);
-        score_chunk<T, D, G, false>(kbase, rs, wv.rope, j0, n, identity, par, C, tv.scale, qrot, s,
-                                    key, CH);
-        for (int i = threadIdx.x; i < n; i += kThreads) ulist[i] = i;
-        __syncthreads();
-        float* outp = part + (int64_t)(NL * wv.SPL + split) * G * (D + 2);
-        if (n == 0) write_empty_partial(outp, G, D);
-        else softmax_partial<T, D, G>(vbase, rs, j0, ulist, n, identity, par, C, s, CH, red, misc, outp);
-        if (split == 0 && threadIdx.x == 0) {
-            cnt_ws[0] = nA;
-            if (cnt_usr) cnt_usr[0] = nA;
-        }
-        return;
-    }
-
-    int32_t* sel_ws = wv.sel + ((int64_t)unit * NL + (level - 1)) * k;
-    int32_t* sel_usr = qv.sel_out ? qv.sel_out + (((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k
-                                  : nullptr;
-    float* outp = part + (int64_t)((level - 1) * wv.SPL + split) * G * (D + 2);
-    if (split == 0 && threadIdx.x == 0) {
+    const int p_q = nA - 1;
+    // scored entries: all of A^(0); at levels >= 1 all but the current entry nA-1
+    const int n_sc = L0 ? max(0, j1 - j0) : max(0, min(j1, nA - 1) - j0);
+    if (!L0 && split == 0 && threadIdx.x == 0) {
         cnt_ws[level] = nA;
         if (cnt_usr) cnt_usr[level] = nA;
     }
-    if (nA <= k) {
-        // everything selected, no summaries (cannot happen below the first scored
-        // level for k, C >= 2, kept for completeness)
+    int32_t* sel_ws = L0 ? nullptr : wv.sel + ((int64_t)unit * NL + (level - 1)) * k;
+    int32_t* sel_usr = (L0 || !qv.sel_out)
+                           ? nullptr
+                           : qv.sel_out + (((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k;
+    float* outp = part + (int64_t)((L0 ? NL * wv.SPL : (level - 1) * wv.SPL) + split) * G * (D + 2);
+    if (!L0 && nA <= k) {
+        // everything selected, no summaries (not reachable below the first scored
+        // level when k, C >= 2; kept for completeness)
         if (split == 0) {
             for (int i = threadIdx.x; i < k; i += kThreads) {
                 int v = -1;
-                if (i < nA) v = identity ? i : C * par[i / C] + (i % C);
+                if (i < nA) v = identity ? i : C * par[cdiv(i, C, lgC)] + cmod(i, C, lgC);
                 if (i < nA) sel_ws[i] = v;
                 if (sel_usr) sel_usr[i] = v;
             }
@@ -504,127 +820,147 @@ __global__ void __launch_bounds__(kThreads) level_kernel(TreeView tv, WorkView w
         return;
     }
 
-    // 1. score the chunk (the current entry nA-1 is never scored)
-    const int n_sc = max(0, min(j1, nA - 1) - j0);
-    score_chunk<T, D, G, true>(kbase, rs, wv.rope, j0, n_sc, identity, par, C, tv.scale, qrot, s,
-                               key, CH);
-    __syncthreads();
+    // ---- the warp's parent groups and their blocks (K then V) ----
+    const int P = (j1 > j0) ? cdiv(j1 - j0 + C - 1, C, lgC) : 0;
+    const int nw = warp < P ? (P - warp + kWarps - 1) / kWarps : 0;
+    const WarpRing R{ring + (size_t)warp * nsw * slot_bytes, bars + warp * nsw, nsw, slot_bytes,
+                     wv.status};
+    auto group_first = [&](int jb) -> int64_t {
+        return identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
+    };
+    auto issue = [&](int q) {
+        const int i = q < nw ? q : q - nw;
+        const int jb = j0 + (warp + kWarps * i) * C;
+        ring_issue<T, D>(R, q, q < nw ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
+    };
+    if (lane == 0)
+        for (int q = 0; q < nsw && q < 2 * nw; ++q) issue(q);
 
-    // 2a. local top-(k-1)
-    block_topk_rank(key, n_sc, K1, rank, hist, misc);
-    for (int i = threadIdx.x; i < n_sc; i += kThreads) {
-        const int r = rank[i];
-        if (r >= 0) { lkey[r] = key[i]; lidx[r] = j0 + i; }
+    // 1. scores of the chunk
+    for (int i = 0; i < nw; ++i) {
+        const unsigned char* blk = ring_wait(R, i);
+        const int jb = j0 + (warp + kWarps * i) * C;
+        const int nch = min(C, j0 + n_sc - jb);
+        if (nch > 0)
+            score_parent<T, D, G, !L0>(blk, jb, j0, nch, group_first(jb), wv.rope, p_q, rc4, qsm,
+                                       tv.scale, s, key, nodes, CH);
+        __syncwarp();
+        if (lane == 0 && i + nsw < 2 * nw) issue(i + nsw);
     }
-    if (threadIdx.x == 0) misc[40] = min(n_sc, K1);
-    __syncthreads();
-
-    // 2b. exchange local lists across the cluster, merge in list order
-    cg::cluster_group cluster = cg::this_cluster();
-    const int csize = (int)cluster.num_blocks();
-    const int crank = (int)cluster.block_rank();
-    cluster.sync();
-    int M = 0, off_self = 0;
-    for (int r = 0; r < csize; ++r) {
-        const int* rn = cluster.map_shared_rank(misc + 40, r);
-        const int nr = *rn;
-        if (r == crank) off_self = M;
-        const uint32_t* rk = cluster.map_shared_rank(lkey, r);
-        const int* ri = cluster.map_shared_rank(lidx, r);
-        for (int i = threadIdx.x; i < nr; i += kThreads) {
-            mkey[M + i] = rk[i];
-            midx[M + i] = ri[i];
-        }
-        M += nr;
-    }
-    cluster.sync();   // every CTA has finished reading remote lists
-
-    // 2c. global top-(k-1) over the merged lists; ranks in list order
-    block_topk_rank(mkey, M, K1, rank, hist, misc);
     for (int i = threadIdx.x; i < n_sc; i += kThreads) flag[i] = 0;
-    __syncthreads();
-    const int n_self = misc[40];
-    for (int i = threadIdx.x; i < n_self; i += kThreads) {
-        const int r = rank[off_self + i];
-        if (r >= 0) {
-            const int j = midx[off_self + i];
-            const int node = identity ? j : C * par[j / C] + (j % C);
-            sel_ws[r] = node;
-            if (sel_usr) sel_usr[r] = node;
-            flag[j - j0] = 1;
-        }
-    }
-    if (crank == 0 && threadIdx.x == 0) {
-        sel_ws[K1] = (int)a[level];
-        if (sel_usr) sel_usr[K1] = (int)a[level];
-    }
-    __syncthreads();
 
-    // 3. summaries: unselected scored entries of this chunk
-    int cu = 0;
-    const int ipt = (n_sc + kThreads - 1) / kThreads;
-    const int i0 = threadIdx.x * ipt, i1 = min(n_sc, i0 + ipt);
-    for (int i = i0; i < i1; ++i) cu += (flag[i] == 0);
-    int nu;
-    int off = block_excl_scan(cu, misc + 2, nu);
-    for (int i = i0; i < i1; ++i)
-        if (flag[i] == 0) ulist[off++] = i;
-    __syncthreads();
-    if (nu == 0) write_empty_partial(outp, G, D);
-    else softmax_partial<T, D, G>(vbase, rs, j0, ulist, nu, identity, par, C, s, CH, red, misc, outp);
-}
-
-// ----------------------------------------------------------------------------
-// combine: log-sum-exp merge of every valid partial into the output
-// ----------------------------------------------------------------------------
-template <typename T, int D, int G>
-__global__ void combine_kernel(TreeView tv, WorkView wv, QueryView qv) {
-    const int unit = blockIdx.x;
-    const int qloc = unit / tv.Hkv, kvh = unit % tv.Hkv;
-    int b, gq;
-    int64_t t;
-    const bool valid = query_pos(qv, wv, qloc, b, t, gq);
-    T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
-    if (!valid) {
-        for (int i = threadIdx.x; i < G * D; i += blockDim.x) out[i] = store_round_f<T>(0.f);
-        if (qv.mode == 1 && threadIdx.x == 0) set_status(wv.status, kStatusBadQuery);
-        return;
-    }
-    int64_t a[kMaxLevels];
-    const int lstar = first_scored_level(t, tv.C, tv.k, a);
-    const float* P = wv.part + (int64_t)unit * wv.NSLOT * G * (D + 2);
-    const int n_lvl_slots = lstar * wv.SPL;
-    const int s0 = wv.NL * wv.SPL;
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-        const int g = i / D, d = i % D;
-        float M = -INFINITY;
-        for (int sl = 0; sl < n_lvl_slots; ++sl) M = fmaxf(M, P[(sl * G + g) * (D + 2) + D]);
-        for (int sl = s0; sl < s0 + wv.NS0; ++sl) M = fmaxf(M, P[(sl * G + g) * (D + 2) + D]);
-        float L = 0.f, O = 0.f;
-        for (int sl = 0; sl < n_lvl_slots + wv.NS0; ++sl) {
-            const int slot = sl < n_lvl_slots ? sl : s0 + (sl - n_lvl_slots);
-            const float* rec = P + (slot * G + g) * (D + 2);
-            const float l = rec[D + 1];
-            if (l > 0.f) {
-                const float w = __expf(rec[D] - M);
-                L += w * l;
-                O += w * rec[d];
-            }
+    if (!L0) {
+        // 2. every CTA's keys in list order (list position = merged index)
+        cg::cluster_group cluster = cg::this_cluster();
+        const int csize = (int)cluster.num_blocks();
+        const int crank = (int)cluster.block_rank();
+        cluster.sync();
+        const int M = nA - 1;
+        for (int r = 0; r < csize; ++r) {
+            const int lo = r * chunk, hi = min(M, lo + chunk);
+            if (hi <= lo) break;
+            const uint32_t* rk = cluster.map_shared_rank(key, r);
+            for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
         }
-        out[i] = store_round_f<T>(L > 0.f ? O / L : 0.f);
+        cluster_arrive();   // remote reads done; matched by cluster_wait() before exit
+        __syncthreads();
+
+        // 3. exact top-(k-1) over all M keys; this CTA writes S for its entries
+        const T* nk;
+        const T* nv;
+        int64_t nrs;
+        if (level == 1) {
+            nk = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
+            nv = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
+            nrs = tv.s_t;
+        } else {
+            nk = level_k<T>(tv, level - 1, b, kvh);
+            nv = level_v<T>(tv, level - 1, b, kvh);
+            nrs = D;
+        }
+        if (K1 > 0)   // k = 1: only the current node is selected
+            select_topk(mkey, M, K1, hist, samp, misc, j0, j0 + n_sc, [&](int i, int r) {
+                const int node = nodes[i - j0];
+                sel_ws[r] = node;
+                if (sel_usr) sel_usr[r] = node;
+                flag[i - j0] = 1;
+                // the children of a selected node are the next level's rows
+                prefetch_children<T, D>(nk, nv, nrs, (int64_t)C * node, C);
+            });
+        if (crank == 0 && threadIdx.x == 0) {
+            const int64_t cur = apow(t, level, C, lgC);
+            sel_ws[K1] = (int)cur;
+            if (sel_usr) sel_usr[K1] = (int)cur;
+            prefetch_children<T, D>(nk, nv, nrs, (int64_t)C * cur,
+                                    (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1));
+        }
+        __syncthreads();
+    }
+
+    // 4. softmax partial over the unselected (level) or all (level 0) entries
+    float lsum[G];
+    // (scratch: the histogram area; the ring, and so red, still holds V blocks)
+    softmax_weights<G>(s, n_sc, L0 ? nullptr : flag, CH, reinterpret_cast<float*>(hist), fm, lsum);
+    float2 acc[G][V2];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < V2; ++e) acc[g][e] = make_float2(0.f, 0.f);
+    for (int i = 0; i < nw; ++i) {
+        const int q = nw + i;
+        const unsigned char* blk = ring_wait(R, q);
+        const int jb = j0 + (warp + kWarps * i) * C;
+        const int nrow = min(C, j0 + n_sc - jb);
+        if (nrow > 0 && fm[0] > -INFINITY)
+            accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
+        __syncwarp();
+        if (lane == 0 && q + nsw < 2 * nw) issue(q + nsw);
+    }
+    __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
+    finish_partial<T, D, G>(acc, lsum, fm, red, outp);
+
+    if (L0) {
+        if (split == 0 && threadIdx.x == 0) {
+            cnt_ws[0] = nA;
+            if (cnt_usr) cnt_usr[0] = nA;
+        }
+        // the last CTA of this unit to finish merges all of the unit's partials
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            misc[kMiscLast] = (atomicAdd(&wv.ucnt[unit], 1u) == (unsigned)nsplit - 1) ? 1 : 0;
+        __syncthreads();
+        if (misc[kMiscLast]) {
+            __threadfence();
+            T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
+            combine_unit<T, D, G>(part, lstar, wv.SPL, wv.NS0, NL, out, red,
+                                  reinterpret_cast<float*>(misc + kMiscFloat + 8));
+            if (threadIdx.x == 0) wv.ucnt[unit] = 0u;
+        }
+    } else {
+        cluster_wait();
     }
 }
 
 // ----------------------------------------------------------------------------
 // host side
 // ----------------------------------------------------------------------------
+static inline int chunk_cap(int k, int splits, int C) { return ((k + splits - 1) / splits) * C; }
+
+// blocks in flight per warp: two when a parent group is at most 4 KB
+static inline int slots_per_warp(int C, int D, int esize) { return C * D * esize <= 4096 ? 2 : 1; }
+
+template <typename T, int D, int G>
+static size_t level_smem(int C, int k, int splits, bool l0) {
+    const int CH = chunk_cap(k, splits, C);
+    const int nsw = slots_per_warp(C, D, (int)sizeof(T));
+    return smem_layout(G, D, CH, k, C, l0 ? 0 : C * k, kWarps * nsw * C * D * (int)sizeof(T)).total;
+}
+
 template <typename T, int D, int G>
 static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
-    const int ck = C * k;
-    const int CH = (ck + SPL - 1) / SPL;
-    const int CH0 = (ck + NS0 - 1) / NS0;
-    const size_t sm = smem_layout(G, D, CH, k, SPL).total;
-    const size_t sm0 = smem_layout(G, D, CH0, k, 1).total;
+    const size_t sm = level_smem<T, D, G>(C, k, SPL, false);
+    const size_t sm0 = level_smem<T, D, G>(C, k, NS0, true);
     if (sm > 227 * 1024 || sm0 > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(level_kernel<T, D, G, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -641,11 +977,11 @@ static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
 template <typename T, int D, int G>
 static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                       cudaStream_t s, const ProfHook* prof) {
-    const int ck = tv.C * tv.k;
-    const int CH = (ck + wv.SPL - 1) / wv.SPL;
-    const int CH0 = (ck + wv.NS0 - 1) / wv.NS0;
-    const size_t sm = smem_layout(G, D, CH, tv.k, wv.SPL).total;
-    const size_t sm0 = smem_layout(G, D, CH0, tv.k, 1).total;
+    const int CH = chunk_cap(tv.k, wv.SPL, tv.C), CH0 = chunk_cap(tv.k, wv.NS0, tv.C);
+    const int NA = tv.C * tv.k;
+    const int nsw = slots_per_warp(tv.C, D, (int)sizeof(T));
+    const size_t sm = level_smem<T, D, G>(tv.C, tv.k, wv.SPL, false);
+    const size_t sm0 = level_smem<T, D, G>(tv.C, tv.k, wv.NS0, true);
     const unsigned units = (unsigned)(qv.nq * tv.Hkv);
     for (int level = wv.NL; level >= 1; --level) {
         cudaLaunchConfig_t cfg = {};
@@ -661,18 +997,15 @@ static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, co
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         prof_mark(prof, level, true, s);
-        cudaError_t e = cudaLaunchKernelEx(&cfg, level_kernel<T, D, G, false>, tv, wv, qv, level, CH);
+        cudaError_t e =
+            cudaLaunchKernelEx(&cfg, level_kernel<T, D, G, false>, tv, wv, qv, level, CH, NA, nsw);
         prof_mark(prof, level, false, s);
         if (e != cudaSuccess) return e;
     }
     prof_mark(prof, 0, true, s);
-    level_kernel<T, D, G, true><<<dim3((unsigned)wv.NS0, units), kThreads, sm0, s>>>(tv, wv, qv, 0, CH0);
+    level_kernel<T, D, G, true><<<dim3((unsigned)wv.NS0, units), kThreads, sm0, s>>>(tv, wv, qv, 0,
+                                                                                    CH0, 0, nsw);
     prof_mark(prof, 0, false, s);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    prof_mark(prof, -2, true, s);
-    combine_kernel<T, D, G><<<units, 128, 0, s>>>(tv, wv, qv);
-    prof_mark(prof, -2, false, s);
     return cudaGetLastError();
 }
 
@@ -712,11 +1045,6 @@ cudaError_t prepare_kernels(int dtype, int D, int G, int SPL, int NS0, int C, in
 cudaError_t launch_select_attend(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                  int dtype, cudaStream_t s, const ProfHook* prof) {
     RECSA_DISPATCH_TDG(dtype, tv.D, tv.G, select_attend_impl, tv, wv, qv, s, prof);
-}
-
-size_t select_smem_bytes(int G, int D, int C, int k, int spl) {
-    const int ck = C * k;
-    return smem_layout(G, D, (ck + spl - 1) / spl, k, spl).total;
 }
 
 }  // namespace recsa

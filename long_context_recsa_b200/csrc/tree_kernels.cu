@@ -112,10 +112,12 @@ __device__ __forceinline__ void level_rows(const TreeView& tv, int l, int b, int
 // ----------------------------------------------------------------------------
 // workspace initialisation: status, lengths, RoPE table
 // ----------------------------------------------------------------------------
-__global__ void init_workspace_kernel(WorkView wv, int B, int D, double base) {
+__global__ void init_workspace_kernel(WorkView wv, TreeView tv, int B, int D, double base) {
     const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (gid == 0) *wv.status = 0u;
     if (gid < B) { wv.lens[gid] = 0; wv.done[gid] = 0u; }
+    if (blockIdx.x == 0) fill_alpha(tv.w, tv.C, const_cast<double*>(wv.alpha));
+    for (int64_t i = gid; i < wv.nunits; i += (int64_t)gridDim.x * blockDim.x) wv.ucnt[i] = 0u;
     const int half = D / 2;
     const int64_t total = (int64_t)wv.ck * half;
     for (int64_t i = gid; i < total; i += (int64_t)gridDim.x * blockDim.x) {
@@ -135,7 +137,7 @@ cudaError_t launch_init_workspace(const TreeView& tv, const WorkView& wv, double
     int blocks = (int)((total + 255) / 256);
     if (blocks < 1) blocks = 1;
     if (blocks > 4096) blocks = 4096;
-    init_workspace_kernel<<<blocks, 256, 0, s>>>(wv, tv.B, tv.D, rope_base);
+    init_workspace_kernel<<<blocks, 256, 0, s>>>(wv, tv, tv.B, tv.D, rope_base);
     return cudaGetLastError();
 }
 
@@ -153,12 +155,9 @@ __global__ void set_lengths_kernel(WorkView wv, Lengths64 L, int B) {
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256) build_pass_kernel(TreeView tv, WorkView wv, int s, int64_t add) {
+__global__ void __launch_bounds__(256, 2) build_pass_kernel(TreeView tv, WorkView wv, int s, int64_t add) {
     __shared__ double alpha[RECSA_MAX_C * RECSA_MAX_C];
-    __shared__ float wsh[RECSA_MAX_C];
-    if (threadIdx.x < RECSA_MAX_C) wsh[threadIdx.x] = tv.w[threadIdx.x];
-    __syncthreads();
-    fill_alpha(wsh, tv.C, alpha);
+    for (int i = threadIdx.x; i < tv.C * tv.C; i += blockDim.x) alpha[i] = wv.alpha[i];
     __syncthreads();
 
     const int bh = blockIdx.y;
@@ -186,10 +185,23 @@ __global__ void __launch_bounds__(256) build_pass_kernel(TreeView tv, WorkView w
     level_rows<T>(tv, s, b, h, sk, sv, rs);
     T* k1 = level_k<T>(tv, s + 1, b, h);
     T* v1 = level_v<T>(tv, s + 1, b, h);
+    const int lane = threadIdx.x & 31;
+    constexpr uint32_t kRow = D * sizeof(T);
     for (int c1 = 0; c1 < C; ++c1) {
         const int64_t i1 = p2 * C + c1;
         if (i1 >= n_s1) break;
         const int m = (int)imin64(C, n_s - i1 * C);
+        // rows of the parent two steps ahead go to L2 while this one is pooled
+        const int64_t ia = i1 + 2;
+        if (lane == 0 && c1 + 2 < C && ia < n_s1) {
+            const int ma = (int)imin64(C, n_s - ia * C);
+            if (rs == D) {
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sk + ia * C * rs),
+                             "r"(ma * kRow) : "memory");
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sv + ia * C * rs),
+                             "r"(ma * kRow) : "memory");
+            }
+        }
         warp_pool_node<T, D>(sk + i1 * C * rs, sv + i1 * C * rs, rs, m, alpha + (m - 1) * C,
                              k1 + i1 * D, v1 + i1 * D, nullptr, nullptr);
     }
@@ -246,7 +258,6 @@ __global__ void __launch_bounds__(128) append1_kernel(TreeView tv, WorkView wv, 
                                                       const T* vnew) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ double alpha[RECSA_MAX_C * RECSA_MAX_C];
-    __shared__ float wsh[RECSA_MAX_C];
     __shared__ int lvl_m[kMaxLevels];
     __shared__ int64_t lvl_i[kMaxLevels];
     __shared__ int n_chain;
@@ -260,24 +271,23 @@ __global__ void __launch_bounds__(128) append1_kernel(TreeView tv, WorkView wv, 
         if (threadIdx.x == 0 && h == 0) set_status(wv.status, kStatusCapacity);
         return;
     }
-    if (threadIdx.x < RECSA_MAX_C) wsh[threadIdx.x] = tv.w[threadIdx.x];
+    for (int i = threadIdx.x; i < C * C; i += blockDim.x) alpha[i] = wv.alpha[i];
     if (threadIdx.x == 0) {
         // ancestors of token L: at level l the node L / C^l with m_l present children
         int64_t n_prev = L + 1;                   // nodes at level l-1
         int64_t idx = L;
         int l = 1;
         while (n_prev > 1 && l < kMaxLevels) {
-            const int64_t i = idx / C;
+            const int64_t i = cdiv64(idx, C, tv.lgC);
             lvl_i[l] = i;
             lvl_m[l] = (int)imin64(C, n_prev - i * C);
-            n_prev = (n_prev + C - 1) / C;
+            n_prev = cdiv64(n_prev + C - 1, C, tv.lgC);
             idx = i;
             ++l;
         }
         n_chain = l - 1;                          // levels 1..n_chain change
     }
     __syncthreads();
-    fill_alpha(wsh, C, alpha);
 
     // staging: slot l holds the C children rows (K then V) of the level-l ancestor
     T* stage = reinterpret_cast<T*>(smem_raw);
@@ -299,7 +309,8 @@ __global__ void __launch_bounds__(128) append1_kernel(TreeView tv, WorkView wv, 
             *reinterpret_cast<uint4*>(stage + (int64_t)C * D + (int64_t)(mm - 1) * D + e * VEC) = vv;
         }
     }
-    // unchanged siblings of every ancestor
+    // unchanged siblings of every ancestor: asynchronous 16-byte copies, all in
+    // flight together, one wait
     for (int l = 1; l <= n_chain; ++l) {
         const T *sk, *sv;
         int64_t rs;
@@ -307,15 +318,18 @@ __global__ void __launch_bounds__(128) append1_kernel(TreeView tv, WorkView wv, 
         const int m = lvl_m[l];
         const int64_t first = lvl_i[l] * C;
         T* slot = stage + (int64_t)(l - 1) * slot_elems;
-        const int per_row = D / VEC;
+        constexpr int per_row = D / VEC;
         for (int e = threadIdx.x; e < (m - 1) * per_row; e += blockDim.x) {
             const int r = e / per_row, c = e % per_row;
-            *reinterpret_cast<uint4*>(slot + (int64_t)r * D + c * VEC) =
-                *reinterpret_cast<const uint4*>(sk + (first + r) * rs + c * VEC);
-            *reinterpret_cast<uint4*>(slot + (int64_t)C * D + (int64_t)r * D + c * VEC) =
-                *reinterpret_cast<const uint4*>(sv + (first + r) * rs + c * VEC);
+            const unsigned dk = (unsigned)__cvta_generic_to_shared(slot + (int64_t)r * D + c * VEC);
+            const unsigned dv = (unsigned)__cvta_generic_to_shared(slot + (int64_t)C * D + (int64_t)r * D + c * VEC);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk),
+                         "l"(sk + (first + r) * rs + c * VEC) : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dv),
+                         "l"(sv + (first + r) * rs + c * VEC) : "memory");
         }
     }
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     if (threadIdx.x < 32) {
         for (int l = 1; l <= n_chain; ++l) {

@@ -199,3 +199,11 @@ def test_host_errors_are_returned_not_launched(R):
     with pytest.raises(R.RecsaError):
         tree.prefill(Q, 88)
     assert tree.recsa_get_status() == R.RECSA_OK
+
+
+@pytest.mark.parametrize("k,L", [(128, 40000), (64, 30000)])
+def test_long_lists_sampled_select(R, k, L):
+    """Lists of 1024-2048 entries: the selection runs on a compact candidate list
+    bounded by a sampled threshold; sets must still be exact."""
+    run_decode_case(R, config_id=17, B=2, Hkv=2, Hq=8, d=128, C=16, k=k, lengths=[L, L - 777],
+                    dtype="bf16", cap=L, n_needles=16)
