@@ -234,13 +234,14 @@ __device__ int block_select_ranks(const uint32_t* keys, int n, uint32_t T, int n
 // compact candidate list (keys >= T0, in list order, packed as (key, position) in
 // mkey); the exact radix select and the ranks then run on that list.  When the
 // estimate misses (fewer than K or more than kCap candidates) the whole list is
-// used.  Both paths give the same result.
+// used.  Both paths give the same result.  mkey holds cap_words words, so the
+// compact list takes at most cap_words / 2 pairs.
 template <typename Fn>
-__device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, uint32_t* sample, int* misc,
-                            int lo, int hi, Fn mark) {
+__device__ void select_topk(uint32_t* mkey, int M, int K, int cap_words, uint32_t* hist,
+                            uint32_t* sample, int* misc, int lo, int hi, Fn mark) {
     constexpr int NS = kThreads;     // sample size, one key per thread
     constexpr int IPT = 16;          // keys per thread held in registers while compacting
-    constexpr int kCap = 2048;       // compact list capacity ((key, position) pairs in mkey)
+    const int kCap = min(2048, cap_words / 2);   // compact list capacity in pairs
     const int tid = threadIdx.x;
     uint32_t T;
     int need_eq, cnt_eq, n0 = 0;
@@ -848,6 +849,9 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
         if (lane == 0 && i + nsw < 2 * nw) issue(i + nsw);
     }
     for (int i = threadIdx.x; i < n_sc; i += kThreads) flag[i] = 0;
+    // every warp's scores are written before any thread reads the chunk's (at
+    // levels >= 1 the cluster barrier below orders them)
+    if (L0) __syncthreads();
 
     if (!L0) {
         // 2. every CTA's keys in list order (list position = merged index)
@@ -879,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
             nrs = D;
         }
         if (K1 > 0)   // k = 1: only the current node is selected
-            select_topk(mkey, M, K1, hist, samp, misc, j0, j0 + n_sc, [&](int i, int r) {
+            select_topk(mkey, M, K1, NA, hist, samp, misc, j0, j0 + n_sc, [&](int i, int r) {
                 const int node = nodes[i - j0];
                 sel_ws[r] = node;
                 if (sel_usr) sel_usr[r] = node;

@@ -248,120 +248,64 @@ __global__ void commit_lengths_kernel(WorkView wv, int B, int64_t add, int64_t c
 }
 
 // ----------------------------------------------------------------------------
-// single-token append: one CTA per (b, h) writes the token and re-pools its
-// ancestors bottom-up.  All unchanged siblings are staged in shared memory with one
-// round of loads; the chain then runs from shared memory.  The last CTA of a
-// sequence advances its length.
+// single-token append, in two kernels.
+//   append_token_kernel: one CTA per sequence writes the new K, V rows of every
+//     KV head at the current length L and advances the length to L + 1.  A decode
+//     at t = L needs nothing else: the ancestors of token L are the current nodes
+//     of every level, which are never scored nor used as summaries.
+//   append_chain_kernel: one CTA per (sequence, KV head) re-pools the ancestors of
+//     token L bottom-up.  The children of every ancestor are staged in shared
+//     memory with one round of asynchronous copies; the chain then runs from
+//     shared memory, each new node becoming the last child of the next one.  It
+//     may run concurrently with a decode and must finish before the next step.
 // ----------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(128) append1_kernel(TreeView tv, WorkView wv, const T* knew,
-                                                      const T* vnew) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ double alpha[RECSA_MAX_C * RECSA_MAX_C];
-    __shared__ int lvl_m[kMaxLevels];
-    __shared__ int64_t lvl_i[kMaxLevels];
-    __shared__ int n_chain;
-    __shared__ bool is_last;
+__global__ void __launch_bounds__(128) append_token_kernel(TreeView tv, WorkView wv, const T* knew,
+                                                           const T* vnew) {
+    const int b = blockIdx.x;
+    const int64_t L = wv.lens[b];
+    if (L + 1 > tv.cap) {
+        if (threadIdx.x == 0) set_status(wv.status, kStatusCapacity);
+        return;
+    }
+    constexpr int VEC = VecOf<T>::N;
+    constexpr int PER_ROW = D / VEC;
+    for (int e = threadIdx.x; e < tv.Hkv * PER_ROW; e += blockDim.x) {
+        const int h = e / PER_ROW, c = e % PER_ROW;
+        const int64_t src = ((int64_t)(b * tv.Hkv + h)) * D + c * VEC;
+        const int64_t dst = b * tv.s_b + h * tv.s_h + L * tv.s_t + c * VEC;
+        *reinterpret_cast<uint4*>(reinterpret_cast<T*>(tv.k0w) + dst) =
+            *reinterpret_cast<const uint4*>(knew + src);
+        *reinterpret_cast<uint4*>(reinterpret_cast<T*>(tv.v0w) + dst) =
+            *reinterpret_cast<const uint4*>(vnew + src);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) wv.lens[b] = L + 1;
+}
 
+template <typename T, int D>
+__global__ void __launch_bounds__(32) append_chain_kernel(TreeView tv, WorkView wv) {
     const int bh = blockIdx.x;
     const int b = bh / tv.Hkv, h = bh % tv.Hkv;
     const int C = tv.C;
-    const int64_t L = wv.lens[b];
-    if (L + 1 > tv.cap) {
-        if (threadIdx.x == 0 && h == 0) set_status(wv.status, kStatusCapacity);
-        return;
-    }
-    for (int i = threadIdx.x; i < C * C; i += blockDim.x) alpha[i] = wv.alpha[i];
-    if (threadIdx.x == 0) {
-        // ancestors of token L: at level l the node L / C^l with m_l present children
-        int64_t n_prev = L + 1;                   // nodes at level l-1
-        int64_t idx = L;
-        int l = 1;
-        while (n_prev > 1 && l < kMaxLevels) {
-            const int64_t i = cdiv64(idx, C, tv.lgC);
-            lvl_i[l] = i;
-            lvl_m[l] = (int)imin64(C, n_prev - i * C);
-            n_prev = cdiv64(n_prev + C - 1, C, tv.lgC);
-            idx = i;
-            ++l;
-        }
-        n_chain = l - 1;                          // levels 1..n_chain change
-    }
-    __syncthreads();
-
-    // staging: slot l holds the C children rows (K then V) of the level-l ancestor
-    T* stage = reinterpret_cast<T*>(smem_raw);
-    const int64_t slot_elems = (int64_t)2 * C * D;
-    constexpr int VEC = VecOf<T>::N;
-    const T* kn = knew + (int64_t)bh * D;
-    const T* vn = vnew + (int64_t)bh * D;
-    T* k0 = reinterpret_cast<T*>(tv.k0w) + (b * tv.s_b + h * tv.s_h);
-    T* v0 = reinterpret_cast<T*>(tv.v0w) + (b * tv.s_b + h * tv.s_h);
-    // the new token: level 0 (global) and its slot in level 1's children
-    for (int e = threadIdx.x; e < D / VEC; e += blockDim.x) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(kn + e * VEC);
-        const uint4 vv = *reinterpret_cast<const uint4*>(vn + e * VEC);
-        *reinterpret_cast<uint4*>(k0 + L * tv.s_t + e * VEC) = kv;
-        *reinterpret_cast<uint4*>(v0 + L * tv.s_t + e * VEC) = vv;
-        if (n_chain >= 1) {
-            const int mm = lvl_m[1];
-            *reinterpret_cast<uint4*>(stage + (int64_t)(mm - 1) * D + e * VEC) = kv;
-            *reinterpret_cast<uint4*>(stage + (int64_t)C * D + (int64_t)(mm - 1) * D + e * VEC) = vv;
-        }
-    }
-    // unchanged siblings of every ancestor: asynchronous 16-byte copies, all in
-    // flight together, one wait
-    for (int l = 1; l <= n_chain; ++l) {
+    const int64_t L = wv.lens[b] - 1;            // the token just appended
+    if (L < 0) return;
+    // ancestors of token L, bottom-up: at level l the node L / C^l, whose m present
+    // children are read from level l-1 (the last of them was written just before)
+    int64_t n_prev = L + 1;                       // nodes at level l-1
+    int64_t idx = L;
+    for (int l = 1; n_prev > 1 && l < kMaxLevels; ++l) {
+        const int64_t i = cdiv64(idx, C, tv.lgC);
+        const int m = (int)imin64(C, n_prev - i * C);
         const T *sk, *sv;
         int64_t rs;
         level_rows<T>(tv, l - 1, b, h, sk, sv, rs);
-        const int m = lvl_m[l];
-        const int64_t first = lvl_i[l] * C;
-        T* slot = stage + (int64_t)(l - 1) * slot_elems;
-        constexpr int per_row = D / VEC;
-        for (int e = threadIdx.x; e < (m - 1) * per_row; e += blockDim.x) {
-            const int r = e / per_row, c = e % per_row;
-            const unsigned dk = (unsigned)__cvta_generic_to_shared(slot + (int64_t)r * D + c * VEC);
-            const unsigned dv = (unsigned)__cvta_generic_to_shared(slot + (int64_t)C * D + (int64_t)r * D + c * VEC);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk),
-                         "l"(sk + (first + r) * rs + c * VEC) : "memory");
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dv),
-                         "l"(sv + (first + r) * rs + c * VEC) : "memory");
-        }
-    }
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        for (int l = 1; l <= n_chain; ++l) {
-            const int m = lvl_m[l];
-            const T* slot = stage + (int64_t)(l - 1) * slot_elems;
-            T* nk = nullptr;
-            T* nv = nullptr;
-            if (l < n_chain) {                     // the new node is the last child above
-                T* up = stage + (int64_t)l * slot_elems;
-                const int mu = lvl_m[l + 1];
-                nk = up + (int64_t)(mu - 1) * D;
-                nv = up + (int64_t)C * D + (int64_t)(mu - 1) * D;
-            }
-            warp_pool_node<T, D>(slot, slot + (int64_t)C * D, D, m, alpha + (m - 1) * C,
-                                 level_k<T>(tv, l, b, h) + lvl_i[l] * D,
-                                 level_v<T>(tv, l, b, h) + lvl_i[l] * D, nk, nv);
-            __syncwarp();
-        }
-    }
-    // advance the length once every head of this sequence is done
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(&wv.done[b], 1u);
-        is_last = (prev == (unsigned)tv.Hkv - 1);
-    }
-    __syncthreads();
-    if (is_last && threadIdx.x == 0) {
-        __threadfence();
-        wv.lens[b] = L + 1;
-        wv.done[b] = 0u;
-        __threadfence();
+        warp_pool_node<T, D>(sk + i * C * rs, sv + i * C * rs, rs, m, wv.alpha + (m - 1) * C,
+                             level_k<T>(tv, l, b, h) + i * D, level_v<T>(tv, l, b, h) + i * D,
+                             nullptr, nullptr);
+        __syncwarp();
+        n_prev = cdiv64(n_prev + C - 1, C, tv.lgC);
+        idx = i;
     }
 }
 
@@ -395,23 +339,10 @@ static cudaError_t build_impl(const TreeView& tv, const WorkView& wv, const int6
     return run_passes<T, D>(tv, wv, 0, s);
 }
 
-constexpr size_t kAppend1MaxSmem = 160 * 1024;
-
-static size_t append1_smem(const TreeView& tv, int esize) {
-    return (size_t)(tv.n_levels) * 2 * tv.C * tv.D * esize;
-}
 
 template <typename T, int D>
 static cudaError_t append_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
                                const void* v_new, int n, cudaStream_t s, const ProfHook* prof) {
-    const size_t sm = append1_smem(tv, (int)sizeof(T));
-    if (n == 1 && sm <= kAppend1MaxSmem) {
-        prof_mark(prof, -1, true, s);
-        append1_kernel<T, D><<<tv.B * tv.Hkv, 128, sm, s>>>(
-            tv, wv, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new));
-        prof_mark(prof, -1, false, s);
-        return cudaGetLastError();
-    }
     const int per_row = D / VecOf<T>::N;
     int64_t blocks = ((int64_t)n * per_row + 255) / 256;
     if (blocks > 1024) blocks = 1024;
@@ -427,6 +358,22 @@ static cudaError_t append_impl(const TreeView& tv, const WorkView& wv, const voi
     return cudaGetLastError();
 }
 
+template <typename T, int D>
+static cudaError_t append_token_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
+                                     const void* v_new, cudaStream_t s, const ProfHook* prof) {
+    prof_mark(prof, -1, true, s);
+    append_token_kernel<T, D><<<tv.B, 128, 0, s>>>(tv, wv, reinterpret_cast<const T*>(k_new),
+                                                   reinterpret_cast<const T*>(v_new));
+    prof_mark(prof, -1, false, s);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t append_chain_impl(const TreeView& tv, const WorkView& wv, cudaStream_t s) {
+    append_chain_kernel<T, D><<<tv.B * tv.Hkv, 32, 0, s>>>(tv, wv);
+    return cudaGetLastError();
+}
+
 #define RECSA_DISPATCH_TD(dtype, D, FN, ...)                                              \
     do {                                                                                  \
         if ((dtype) == RECSA_BF16 && (D) == 128) return FN<__nv_bfloat16, 128>(__VA_ARGS__); \
@@ -437,11 +384,8 @@ static cudaError_t append_impl(const TreeView& tv, const WorkView& wv, const voi
     } while (0)
 
 template <typename T, int D>
-static cudaError_t prepare_tree_impl(const TreeView& tv) {
-    const size_t sm = append1_smem(tv, (int)sizeof(T));
-    if (sm > kAppend1MaxSmem) return cudaSuccess;     // multi-pass path is used instead
-    return cudaFuncSetAttribute(append1_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sm);
+static cudaError_t prepare_tree_impl(const TreeView&) {
+    return cudaSuccess;
 }
 
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype) {
@@ -458,6 +402,17 @@ cudaError_t launch_set_lengths(const WorkView& wv, const int64_t* lengths, int B
 cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
                          int dtype, cudaStream_t s) {
     RECSA_DISPATCH_TD(dtype, tv.D, build_impl, tv, wv, lengths, s);
+}
+
+bool single_append_supported(const TreeView&, int) { return true; }
+
+cudaError_t launch_append_token(const TreeView& tv, const WorkView& wv, const void* k_new,
+                                const void* v_new, int dtype, cudaStream_t s, const ProfHook* prof) {
+    RECSA_DISPATCH_TD(dtype, tv.D, append_token_impl, tv, wv, k_new, v_new, s, prof);
+}
+
+cudaError_t launch_append_chain(const TreeView& tv, const WorkView& wv, int dtype, cudaStream_t s) {
+    RECSA_DISPATCH_TD(dtype, tv.D, append_chain_impl, tv, wv, s);
 }
 
 cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
