@@ -130,14 +130,8 @@ RECSA_API recsa_status recsa_build(recsa_tree* tree, const int64_t* lengths, voi
  * by append(n) is bitwise equal to build(L+n)), and L grows by n.  If L + n would
  * exceed capacity the sequence is left unchanged and the status word records
  * RECSA_E_CAPACITY (the host also rejects this synchronously while its own copy
- * of the lengths is current, i.e. outside graph replays).
- * With n == 1 the new rows and lengths are written on `stream`, and the ancestor
- * re-pooling runs on an internal stream of the handle, forked from `stream` by an
- * event: a decode that follows overlaps it (it reads no ancestor of the new
- * token).  The next recsa_decode, recsa_prefill_chunk, recsa_append, recsa_build
- * or recsa_get_status on the handle makes its stream wait for it, so a stream
- * capture that contains an append must also contain one of those calls after it.
- * The handle is not thread-safe. */
+ * of the lengths is current, i.e. outside graph replays).  With n == 1 the whole
+ * update (new rows, every ancestor, the length) is one kernel launch. */
 RECSA_API recsa_status recsa_append(recsa_tree* tree, const void* k_new, const void* v_new, int32_t n,
                           void* stream);
 

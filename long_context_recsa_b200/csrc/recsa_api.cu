@@ -169,19 +169,7 @@ struct recsa_tree {
     WorkView wv;
     int64_t host_len[RECSA_MAX_BATCH];
     ProfHook prof;
-    // single-token appends re-pool the ancestors on a side stream; the next call
-    // that needs them joins it
-    cudaStream_t side;
-    cudaEvent_t ev_fork, ev_join;
-    bool chain_pending;
 };
-
-// Make `stream` wait for an ancestor update still running on the side stream.
-static recsa_status join_chain(recsa_tree* t, cudaStream_t stream) {
-    if (!t->chain_pending) return RECSA_OK;
-    t->chain_pending = false;
-    return cudaStreamWaitEvent(stream, t->ev_join, 0) == cudaSuccess ? RECSA_OK : RECSA_E_CUDA;
-}
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -280,14 +268,8 @@ recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t 
 
     cudaError_t e = prepare_kernels(cfg->dtype, L.D, L.G, L.SPL, L.NS0, cfg->C, cfg->k);
     if (e == cudaSuccess) e = prepare_tree_kernels(tv, cfg->dtype);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&t->side, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t->ev_fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t->ev_join, cudaEventDisableTiming);
     if (e == cudaSuccess) e = launch_init_workspace(tv, wv, cfg->rope_base, (cudaStream_t)stream);
     if (e != cudaSuccess) {
-        if (t->ev_join) cudaEventDestroy(t->ev_join);
-        if (t->ev_fork) cudaEventDestroy(t->ev_fork);
-        if (t->side) cudaStreamDestroy(t->side);
         free(t);
         return RECSA_E_CUDA;
     }
@@ -299,7 +281,6 @@ recsa_status recsa_build(recsa_tree* t, const int64_t* lengths, void* stream) {
     if (!t || !lengths) return RECSA_E_INVAL;
     for (int b = 0; b < t->B; ++b)
         if (lengths[b] < 0 || lengths[b] > t->cap) return RECSA_E_CAPACITY;
-    if (join_chain(t, (cudaStream_t)stream) != RECSA_OK) return RECSA_E_CUDA;
     cudaError_t e = launch_build(t->tv, t->wv, lengths, t->cfg.dtype, (cudaStream_t)stream);
     if (e != cudaSuccess) return RECSA_E_CUDA;
     for (int b = 0; b < t->B; ++b) t->host_len[b] = lengths[b];
@@ -313,16 +294,9 @@ recsa_status recsa_append(recsa_tree* t, const void* k_new, const void* v_new, i
     for (int b = 0; b < t->B; ++b)
         if (t->host_len[b] + n > t->cap) return RECSA_E_CAPACITY;
     const cudaStream_t s = (cudaStream_t)stream;
-    // the previous step's ancestors must be complete before this step touches them
-    if (join_chain(t, s) != RECSA_OK) return RECSA_E_CUDA;
     cudaError_t e;
-    if (n == 1 && single_append_supported(t->tv, t->L.esize)) {
-        e = launch_append_token(t->tv, t->wv, k_new, v_new, t->cfg.dtype, s, &t->prof);
-        if (e == cudaSuccess) e = cudaEventRecord(t->ev_fork, s);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(t->side, t->ev_fork, 0);
-        if (e == cudaSuccess) e = launch_append_chain(t->tv, t->wv, t->cfg.dtype, t->side);
-        if (e == cudaSuccess) e = cudaEventRecord(t->ev_join, t->side);
-        if (e == cudaSuccess) t->chain_pending = true;
+    if (n == 1) {
+        e = launch_append_one(t->tv, t->wv, k_new, v_new, t->cfg.dtype, s, &t->prof);
     } else {
         e = launch_append(t->tv, t->wv, k_new, v_new, n, t->cfg.dtype, s, &t->prof);
     }
@@ -347,9 +321,7 @@ recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_
     qv.nq = t->B;
     cudaError_t e =
         launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof);
-    if (e != cudaSuccess) return RECSA_E_CUDA;
-    // the ancestor update of the last append ran alongside; join it here
-    return join_chain(t, (cudaStream_t)stream);
+    return e == cudaSuccess ? RECSA_OK : RECSA_E_CUDA;
 }
 
 recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int32_t n, void* O,
@@ -374,12 +346,11 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
             launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof);
         if (e != cudaSuccess) return RECSA_E_CUDA;
     }
-    return join_chain(t, (cudaStream_t)stream);
+    return RECSA_OK;
 }
 
 recsa_status recsa_get_status(recsa_tree* t, void* stream) {
     if (!t) return RECSA_E_INVAL;
-    if (join_chain(t, (cudaStream_t)stream) != RECSA_OK) return RECSA_E_CUDA;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RECSA_E_CUDA;
     uint32_t v = 0;
     if (cudaMemcpy(&v, t->wv.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
@@ -432,10 +403,6 @@ recsa_status recsa_set_profile_events(recsa_tree* t, int32_t which, void* start,
 
 recsa_status recsa_tree_free(recsa_tree* t) {
     if (!t) return RECSA_E_INVAL;
-    cudaStreamSynchronize(t->side);
-    cudaEventDestroy(t->ev_join);
-    cudaEventDestroy(t->ev_fork);
-    cudaStreamDestroy(t->side);
     free(t);
     return RECSA_OK;
 }

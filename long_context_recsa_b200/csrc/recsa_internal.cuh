@@ -286,11 +286,9 @@ cudaError_t launch_init_workspace(const TreeView& tv, const WorkView& wv, double
                                   cudaStream_t s);
 cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
                          int dtype, cudaStream_t s);
-bool single_append_supported(const TreeView& tv, int esize);
-cudaError_t launch_append_token(const TreeView& tv, const WorkView& wv, const void* k_new,
-                                const void* v_new, int dtype, cudaStream_t s,
-                                const ProfHook* prof = nullptr);
-cudaError_t launch_append_chain(const TreeView& tv, const WorkView& wv, int dtype, cudaStream_t s);
+cudaError_t launch_append_one(const TreeView& tv, const WorkView& wv, const void* k_new,
+                              const void* v_new, int dtype, cudaStream_t s,
+                              const ProfHook* prof = nullptr);
 cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
                           const void* v_new, int n, int dtype, cudaStream_t s,
                           const ProfHook* prof = nullptr);
