@@ -27,6 +27,31 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
+
+# DRAM bytes (read + write) per launch of the level-1 select/attend kernel from one
+# ncu capture at batch 1 (profiles/level_kernels_decode524k_b1.md); a launch covers
+# batch x 8 independent units, so the batch-B figure is B times this.  Valid only
+# for the kernel sources it was taken from: any edit to them turns it into null.
+TRAFFIC_LEVEL1_B1 = {"bytes": 33_760_256 + 768,
+                     "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
+                                 "long_context_recsa_b200/csrc/recsa_internal.cuh"],
+                     "sha256": "205cddb9d634061dab3e189d15fb56466644d673033cf909e4118b25db02ea3c"}
+
+
+def captured_traffic(kernel: str, batch: int):
+    """Per-launch DRAM traffic of `kernel` at this batch, or None when no capture of
+    the current sources exists."""
+    import hashlib
+    if kernel != "level1_kernel":
+        return None
+    h = hashlib.sha256()
+    here = os.path.dirname(os.path.abspath(__file__))
+    for f in TRAFFIC_LEVEL1_B1["sources"]:
+        with open(os.path.join(here, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != TRAFFIC_LEVEL1_B1["sha256"]:
+        return None
+    return TRAFFIC_LEVEL1_B1["bytes"] * batch
 HBM_NOMINAL_GBS = 8000.0
 
 # workload: 524K decode, B = 4 (and the 4096-query prefill chunk at 524K)
@@ -205,7 +230,7 @@ def run_ours(args):
     out = torch.empty_like(qst)
     cnt = torch.zeros(B, Hkv, tree.n_sel_levels + 1, dtype=torch.int32, device=dev)
     prof_ev = {}
-    for which in [0] + list(range(1, tree.n_sel_levels + 1)) + [-1, -2]:
+    for which in [0] + list(range(1, tree.n_sel_levels + 1)) + [-1]:
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(); b_.record()
         prof_ev[which] = (a, b_)
@@ -224,7 +249,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    launches_per_step = 1 + tree.n_sel_levels + 2
+    launches_per_step = 1 + tree.n_sel_levels + 1   # append, levels n..1, level 0
     step_ms, kern_ms = [], {w: [] for w in prof_ev}
     whiches = list(prof_ev)
 
@@ -265,7 +290,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: K,V,q,new k/v ~ N(0,1) seeded, resident in HBM",
-        "config": {"workload": "decode 524K ctx, batch 4, append 1 token/seq/step, "
+        "config": {"workload": f"decode 524K ctx, batch {B}, append 1 token/seq/step, "
                                "Hq=32 Hkv=8 d=128 C=16 k=256 bf16",
                    "seq_len": L, "global_batch": B * ws, "parallelism": f"replicas x{ws}",
                    "l2": "flushed (256 MB write) before every timed step",
@@ -275,11 +300,14 @@ def run_ours(args):
         "hbm_frac_of_measured": round(by_step / (ms / 1e3) / 1e9 / hbm, 4),
         "roofline": {"bound": "hbm", "kernel": f"level{dom}_kernel",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": None,
+                     "frac": round(achieved / hbm, 4),
+                     "traffic": captured_traffic(f"level{dom}_kernel", B),
+                     "traffic_note": "ncu batch-1 capture x batch; includes the L2 prefetch "
+                                     "of the next level's rows (255 x 16 rows x 512 B per unit)",
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": int(dom_bytes),
                      "avg_launch_ms": round(kern_avg[dom], 5)},
-        "kernel_ms": {("append" if w == -1 else "combine" if w == -2 else f"level{w}"):
+        "kernel_ms": {("append" if w == -1 else f"level{w}"):
                       (round(v, 5) if v else None) for w, v in kern_avg.items()},
         "build_524k": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1)},
         "gpu_launches": launches_per_step * args.steps,

@@ -188,7 +188,7 @@ RECSA_API recsa_status recsa_host_lengths(const recsa_tree* tree, int64_t* lengt
  * before the kernel selected by `which` is launched and `stop` just after it:
  *   which = l in [0, n_sel_levels]: the select/attend kernel of level l (0 = the
  *           level-0 attention), in recsa_decode and in each prefill wave;
- *   which = -1: the append kernel(s) of recsa_append;  -2: the combine kernel.
+ *   which = -1: the append kernel(s) of recsa_append.
  * Records use cudaEventRecordExternal, so they also become event nodes when the
  * call is captured in a CUDA graph.  start = stop = NULL clears the hook.
  * No device memory is touched. */

@@ -394,7 +394,7 @@ recsa_status recsa_host_lengths(const recsa_tree* t, int64_t* lengths) {
 
 recsa_status recsa_set_profile_events(recsa_tree* t, int32_t which, void* start, void* stop) {
     if (!t || ((start == nullptr) != (stop == nullptr))) return RECSA_E_INVAL;
-    if (start != nullptr && (which < -2 || which > t->L.NL)) return RECSA_E_INVAL;
+    if (start != nullptr && (which < -1 || which > t->L.NL)) return RECSA_E_INVAL;
     t->prof.which = start ? which : -100;
     t->prof.start = (cudaEvent_t)start;
     t->prof.stop = (cudaEvent_t)stop;
