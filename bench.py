@@ -59,7 +59,7 @@ W = dict(Hq=32, Hkv=8, d=128, C=16, k=256, L=524288, B=4, dtype="bf16", base=1e6
          prefill_q=4096)
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
@@ -70,7 +70,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--batch", type=int, default=4,
                    help="sequences per GPU (the headline workload uses 4)")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 def peaks():
@@ -152,7 +152,10 @@ def step_bytes(counts, k, s_vec, B, Hkv, Hq, d, esize):
     return tot + io, per_level
 
 
-def dist_setup(args):
+def dist_setup(args=None, backend: str = "nccl"):
+    """Rank, world size and local rank from the torchrun environment; one process
+    per GPU over NCCL (gloo for the CPU tests), with a short timeout so that ranks
+    waiting on a lost peer fail instead of hanging."""
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -160,22 +163,46 @@ def dist_setup(args):
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
 
-def max_over_ranks(x, ws):
+def max_over_ranks(x, ws, device: str = "cuda"):
+    """The largest of the ranks' values (the step time every rank reports)."""
     import torch
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def workload_config(B: int, ws: int) -> dict:
+    """The bench's workload, named by what it is (both arms report this)."""
+    return {"workload": f"decode 524K ctx, batch {B}, append 1 token/seq/step, "
+                        "Hq=32 Hkv=8 d=128 C=16 k=256 bf16",
+            "seq_len": W["L"], "global_batch": B * ws, "parallelism": f"replicas x{ws}",
+            "l2": "flushed (256 MB write) before every timed step",
+            "timing": "per-step CUDA events around one graph replay"}
+
+
+def whole_job_value(ms_max: float, ws: int, seqs_per_rank: int) -> float:
+    """Tokens per second of the whole job: every rank decodes its own sequences, one
+    token each per step, and the job's step time is the slowest rank's."""
+    return ws * seqs_per_rank / (ms_max / 1e3)
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own sequences (weak scaling: no rank shares data)."""
+    return base + 7919 * rank
 
 
 def barrier(ws):
@@ -204,7 +231,7 @@ def run_ours(args):
                    rope_base=W["base"], pooler_w=I.pooler_w(C).tolist())
     # inputs resident in HBM before timing (seeded, per rank)
     g = torch.Generator(device=dev)
-    g.manual_seed(I.slice_seed(3, I.STREAM_K, 0, 0) + 7919 * rank)
+    g.manual_seed(rank_seed(I.slice_seed(3, I.STREAM_K, 0, 0), rank))
     K = torch.randn(B, Hkv, cap, d, generator=g, device=dev, dtype=torch.float32).to(dt)
     V = torch.randn(B, Hkv, cap, d, generator=g, device=dev, dtype=torch.float32).to(dt)
     knew = torch.randn(S, B, Hkv, 1, d, generator=g, device=dev, dtype=torch.float32).to(dt)
@@ -276,7 +303,7 @@ def run_ours(args):
         barrier(ws)
     assert tree.recsa_get_status() == R.RECSA_OK
     ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
-    value = ws * B / (ms / 1e3)
+    value = whole_job_value(ms, ws, B)
     counts = cnt.cpu().numpy()
     by_step, per_level = step_bytes(counts, k, d * esize, B, Hkv, Hq, d, esize)
     hbm, peak_kind = peaks()
@@ -290,11 +317,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: K,V,q,new k/v ~ N(0,1) seeded, resident in HBM",
-        "config": {"workload": f"decode 524K ctx, batch {B}, append 1 token/seq/step, "
-                               "Hq=32 Hkv=8 d=128 C=16 k=256 bf16",
-                   "seq_len": L, "global_batch": B * ws, "parallelism": f"replicas x{ws}",
-                   "l2": "flushed (256 MB write) before every timed step",
-                   "timing": "per-step CUDA events around one graph replay"},
+        "config": workload_config(B, ws),
         "bytes_per_step": int(by_step),
         "hbm_frac_of_nominal_8TBs": round(by_step / (ms / 1e3) / 1e9 / HBM_NOMINAL_GBS, 4),
         "hbm_frac_of_measured": round(by_step / (ms / 1e3) / 1e9 / hbm, 4),
@@ -428,7 +451,8 @@ def run_reference(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
-        return
+        return   # the oracle runs on rank 0 only; the other ranks exit without work
+    W["B"] = args.batch
     import numpy as np
     from long_context_recsa_b200 import inputs as I
     from oracle import recsa_oracle as O
@@ -450,8 +474,7 @@ def run_reference(args):
            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(el * Hkv * 1e3, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": "decode 524K ctx, Hq=32 Hkv=8 d=128 C=16 k=256 (oracle sample)",
-                      "seq_len": L},
+           "config": workload_config(W["B"], ws),
            "cpu_baseline": {"value": round(tok_s, 3), "unit": "tok/s", "cores": cores,
                             "kind": "oracle",
                             "sample": "per step: select+attend of one decode query for one "
