@@ -82,6 +82,18 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tf32_peak():
+    """Dense tf32 tensor peak: the measured bf16 burst figure x the nominal tf32/bf16
+    ratio (1.1 / 2.25 PFLOP/s), else the fallback 1.59 PFLOP/s x that ratio."""
+    ratio = 1.1 / 2.25
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]) * ratio, "measured bf16 burst x 1.1/2.25"
+    except Exception:
+        return 1590.0 * ratio, "fallback bf16 x 1.1/2.25"
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle sampling during the timed region."""
 
@@ -413,9 +425,45 @@ def bench_prefill(R, I, cfg, K, V, tree_decode, args, ws, dev, flush):
         times.append(e0.elapsed_time(e1))
     assert pt.recsa_get_status() == R.RECSA_OK
     ms = max_over_ranks(sum(times) / len(times), ws)
-    return {"value": round(ws * nq / (ms / 1e3), 1), "unit": "tok/s", "ms_per_chunk": round(ms, 3),
-            "workload": "4096-query chunk at positions 520192..524287 of a 524288-token tree, "
-                        "batch 1, same shapes", "path": "per-query select/attend kernels"}
+    res = {"value": round(ws * nq / (ms / 1e3), 1), "unit": "tok/s", "ms_per_chunk": round(ms, 3),
+           "workload": "4096-query chunk at positions 520192..524287 of a 524288-token tree, "
+                       "batch 1, same shapes"}
+    if pt.tc_queries > 0:
+        # the top level's tensor-core product: time the chunk's last one with events
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); b_.record()   # torch needs to see them recorded once
+        pt.recsa_set_profile_events(-2, a, b_)
+        pt.recsa_prefill_chunk(Q, L - nq, O)
+        torch.cuda.synchronize()
+        pt.recsa_set_profile_events(-2, None, None)
+        tc_ms = a.elapsed_time(b_)
+        G, d, Hkv, C = W["Hq"] // W["Hkv"], W["d"], W["Hkv"], W["C"]
+        rows = min(pt.tc_queries, nq)
+        t_last = L - 1
+        lt = 0
+        p = t_last
+        while p > 0:
+            p //= C
+            if p >= W["k"]:
+                lt += 1
+            else:
+                break
+        n_nodes = t_last // C ** lt + 1
+        mt, nt = -(-rows * G // 128) * 128, -(-n_nodes // 256) * 256
+        useful = 2.0 * rows * G * n_nodes * d * Hkv
+        executed = 3 * 2.0 * mt * nt * d * Hkv
+        peak, src = tf32_peak()
+        res["path"] = ("top level: one tcgen05 product (split tf32, 3 MMAs) per group of "
+                       f"{pt.tc_queries} rows; lower levels per row")
+        res["tensor_product"] = {
+            "ms_per_launch": round(tc_ms, 4), "level": lt, "rows": rows, "nodes": n_nodes,
+            "useful_tflops": round(useful / (tc_ms / 1e3) / 1e12, 1),
+            "executed_tflops": round(executed / (tc_ms / 1e3) / 1e12, 1),
+            "peak_tflops": round(peak, 1), "peak_source": src,
+            "frac_executed": round(executed / (tc_ms / 1e3) / 1e12 / peak, 3)}
+    else:
+        res["path"] = "per-row select/attend kernels at every level"
+    return res
 
 
 def cpu_baseline(K, V, qs, cfg, R):

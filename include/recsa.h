@@ -153,7 +153,16 @@ RECSA_API recsa_status recsa_decode(recsa_tree* tree, const void* q, void* out, 
  * must already be in the tree (pos0 + n <= L_b).
  *   Q  [batch][n][Hq][d] device;  O [batch][n][Hq][d] device.
  *   sel_out / counts_out as in recsa_decode with batch*n queries (b-major).
- * Each row equals recsa_decode of a tree holding only tokens [0..pos0+i]. */
+ * Each row is the RecSA output of a tree holding only tokens [0..pos0+i].
+ * When the tree was created with max_queries >= 128 (see recsa_tree_info's
+ * tc_queries), the rows of a sequence are taken in groups of up to tc_queries, and
+ * at the first scored level of the group's last row ("Hierarchical Selection",
+ * Eq.3: the list [0..a_t] shared by the group up to each row's cut) the logits of
+ * every row and head against every node come from one tensor-core product
+ * (split-precision tf32, fp32 accumulation).  Rows then match recsa_decode of the
+ * truncated tree up to fp32 rounding of those logits, and their selections agree
+ * except at near-ties.  Otherwise every level is scored per row, and each row is
+ * bitwise equal to that decode. */
 RECSA_API recsa_status recsa_prefill_chunk(recsa_tree* tree, const void* Q, int64_t pos0, int32_t n,
                                  void* O, int32_t* sel_out, int32_t* counts_out, void* stream);
 
@@ -169,6 +178,14 @@ typedef struct {
     int64_t capacity;
     int32_t batch;
     int32_t max_queries;
+    /* tensor-core prefill path (0 when disabled): rows per product, the length of a
+     * logits row, and where the logits of the last product sit in the workspace:
+     * fp32 [tc_queries][Hkv][G][tc_row_stride], scaled by the softmax scale, row
+     * (q, h, g) = that group's row q, KV head h, query head h*G + g; entry j is node
+     * j of the level the product scored.  For diagnostics. */
+    int32_t tc_queries;
+    int32_t tc_row_stride;
+    int64_t tc_logits_offset;
 } recsa_tree_info_t;
 
 RECSA_API recsa_status recsa_tree_info(const recsa_tree* tree, recsa_tree_info_t* info);
@@ -188,7 +205,8 @@ RECSA_API recsa_status recsa_host_lengths(const recsa_tree* tree, int64_t* lengt
  * before the kernel selected by `which` is launched and `stop` just after it:
  *   which = l in [0, n_sel_levels]: the select/attend kernel of level l (0 = the
  *           level-0 attention), in recsa_decode and in each prefill wave;
- *   which = -1: the append kernel(s) of recsa_append.
+ *   which = -1: the append kernel(s) of recsa_append;  -2: the tensor-core product
+ *   of recsa_prefill_chunk (the last one of the call).
  * Records use cudaEventRecordExternal, so they also become event nodes when the
  * call is captured in a CUDA graph.  start = stop = NULL clears the hook.
  * No device memory is touched. */

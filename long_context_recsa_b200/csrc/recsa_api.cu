@@ -9,6 +9,9 @@ namespace recsa {
 
 constexpr int kSplits = 8;    // CTAs (one thread-block cluster) per unit, levels >= 1
 constexpr int kSplits0 = 8;   // CTAs per unit at level 0
+constexpr int kTcMinQueries = 128;   // trees with this many queries get the tensor-core path
+constexpr int kTcQueries = 128;      // prefill rows per tensor-core product
+constexpr int kTcMinRows = 32;       // smaller groups are scored per row
 
 struct Layout {
     int esize, D, G;
@@ -18,6 +21,9 @@ struct Layout {
     size_t level_bytes;
     int NL, SPL, NS0, NSLOT;
     size_t o_status, o_lens, o_done, o_alpha, o_rope, o_sel, o_cnt, o_part, o_ucnt, ws_bytes;
+    // tensor-core prefill buffers (tc_nsub == 0: disabled)
+    int tc_nsub, tc_npad, tc_MB, tc_NB;
+    size_t o_tca_hi, o_tca_lo, o_tcb_hi, o_tcb_lo, o_tclog;
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -92,6 +98,24 @@ static recsa_status compute_layout(const recsa_config* c, int64_t cap, int B, in
     L->o_cnt = w;    w = al256(w + sizeof(int32_t) * (size_t)Qmax * Hkv * (NL + 1));
     L->o_part = w;   w = al256(w + sizeof(float) * (size_t)Qmax * Hkv * L->NSLOT * L->G * (L->D + 2));
     L->o_ucnt = w;   w = al256(w + sizeof(uint32_t) * (size_t)Qmax * Hkv);
+    // tensor-core prefill: trees meant for chunks of queries (max_queries >= 128)
+    L->tc_nsub = 0;
+    L->o_tca_hi = L->o_tca_lo = L->o_tcb_hi = L->o_tcb_lo = L->o_tclog = 0;
+    if (Qmax >= kTcMinQueries && NL >= 1 && (L->D == 64 || L->D == 128)) {
+        const int nsub = kTcQueries < Qmax ? kTcQueries : Qmax;
+        L->tc_nsub = nsub;
+        L->tc_MB = (nsub * L->G + 127) / 128;
+        L->tc_NB = (ck + 255) / 256;
+        L->tc_npad = L->tc_NB * 256;
+        const size_t a_img = (size_t)Hkv * L->tc_MB * (L->D / 32) * 128 * 128;
+        const size_t b_img = (size_t)Hkv * L->tc_NB * (L->D / 32) * 256 * 128;
+        w = (w + 1023) & ~size_t(1023);
+        L->o_tca_hi = w; w = al256(w + a_img);
+        L->o_tca_lo = w; w = al256(w + a_img);
+        L->o_tcb_hi = w; w = al256(w + b_img);
+        L->o_tcb_lo = w; w = al256(w + b_img);
+        L->o_tclog = w;  w = al256(w + sizeof(float) * (size_t)nsub * Hkv * L->G * L->tc_npad);
+    }
     L->ws_bytes = w;
     return RECSA_OK;
 }
@@ -169,6 +193,7 @@ struct recsa_tree {
     WorkView wv;
     int64_t host_len[RECSA_MAX_BATCH];
     ProfHook prof;
+    TcView tc;                 // tensor-core prefill buffers (tc.nsub == 0: none)
 };
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -265,9 +290,23 @@ recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t 
     wv.NS0 = L.NS0;
     wv.NSLOT = L.NSLOT;
     wv.ck = cfg->C * cfg->k;
+    TcView& tc = t->tc;
+    memset(&tc, 0, sizeof(tc));
+    if (L.tc_nsub > 0) {
+        tc.a_hi = (uint32_t*)(ws + L.o_tca_hi);
+        tc.a_lo = (uint32_t*)(ws + L.o_tca_lo);
+        tc.b_hi = (uint32_t*)(ws + L.o_tcb_hi);
+        tc.b_lo = (uint32_t*)(ws + L.o_tcb_lo);
+        tc.logits = (float*)(ws + L.o_tclog);
+        tc.nsub = L.tc_nsub;
+        tc.npad = L.tc_npad;
+        tc.MB = L.tc_MB;
+        tc.NB = L.tc_NB;
+    }
 
     cudaError_t e = prepare_kernels(cfg->dtype, L.D, L.G, L.SPL, L.NS0, cfg->C, cfg->k);
     if (e == cudaSuccess) e = prepare_tree_kernels(tv, cfg->dtype);
+    if (e == cudaSuccess && L.tc_nsub > 0) e = prepare_tc_kernels(L.D);
     if (e == cudaSuccess) e = launch_init_workspace(tv, wv, cfg->rope_base, (cudaStream_t)stream);
     if (e != cudaSuccess) {
         free(t);
@@ -324,14 +363,29 @@ recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_
     return e == cudaSuccess ? RECSA_OK : RECSA_E_CUDA;
 }
 
+// t / C^l and the first scored level of position t (host side of Eq.3's sizes).
+static int64_t host_apow(int64_t t, int l, int C) {
+    for (int i = 0; i < l; ++i) t /= C;
+    return t;
+}
+static int host_first_scored_level(int64_t t, int C, int k) {
+    int lstar = 0, l = 0;
+    for (int64_t p = t; p > 0 && l + 1 < kMaxLevels;) {
+        p /= C;
+        ++l;
+        if (p >= k) lstar = l;
+    }
+    return lstar;
+}
+
 recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int32_t n, void* O,
                                  int32_t* sel_out, int32_t* counts_out, void* stream) {
     if (!t || !Q || !O || n < 1 || pos0 < 0) return RECSA_E_INVAL;
     if (!aligned16(Q) || !aligned16(O)) return RECSA_E_INVAL;
     for (int b = 0; b < t->B; ++b)
         if (pos0 + n > t->host_len[b]) return RECSA_E_CAPACITY;
-    const int total = t->B * n;
-    for (int q0 = 0; q0 < total; q0 += t->Qmax) {
+    const cudaStream_t s = (cudaStream_t)stream;
+    auto base_view = [&]() {
         QueryView qv = {};
         qv.q = Q;
         qv.out = O;
@@ -340,10 +394,40 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
         qv.mode = 1;
         qv.n_per_b = n;
         qv.pos0 = pos0;
+        return qv;
+    };
+    if (t->tc.nsub > 0 && n >= kTcMinRows) {
+        // per sequence, groups of up to tc.nsub rows: the group's first scored level
+        // comes from one tensor-core product, the levels below from the row kernels
+        for (int b = 0; b < t->B; ++b) {
+            for (int i0 = 0; i0 < n; i0 += t->tc.nsub) {
+                const int cnt = n - i0 < t->tc.nsub ? n - i0 : t->tc.nsub;
+                QueryView qv = base_view();
+                qv.q_begin = b * n + i0;
+                qv.nq = cnt;
+                const int64_t t_last = pos0 + i0 + cnt - 1;
+                const int lt = host_first_scored_level(t_last, t->cfg.C, t->cfg.k);
+                if (lt >= 1 && cnt >= kTcMinRows) {
+                    cudaError_t e = launch_prefill_top_tc(t->tv, t->wv, qv, t->tc, lt,
+                                                          host_apow(t_last, lt, t->cfg.C),
+                                                          t->cfg.dtype, s, &t->prof);
+                    if (e != cudaSuccess) return RECSA_E_CUDA;
+                    qv.pre = t->tc.logits;
+                    qv.pre_level = lt;
+                    qv.pre_stride = t->tc.npad;
+                }
+                cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof);
+                if (e != cudaSuccess) return RECSA_E_CUDA;
+            }
+        }
+        return RECSA_OK;
+    }
+    const int total = t->B * n;
+    for (int q0 = 0; q0 < total; q0 += t->Qmax) {
+        QueryView qv = base_view();
         qv.q_begin = q0;
         qv.nq = total - q0 < t->Qmax ? total - q0 : t->Qmax;
-        cudaError_t e =
-            launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof);
+        cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof);
         if (e != cudaSuccess) return RECSA_E_CUDA;
     }
     return RECSA_OK;
@@ -374,6 +458,9 @@ recsa_status recsa_tree_info(const recsa_tree* t, recsa_tree_info_t* info) {
     info->capacity = t->cap;
     info->batch = t->B;
     info->max_queries = t->Qmax;
+    info->tc_queries = t->tc.nsub;
+    info->tc_row_stride = t->tc.npad;
+    info->tc_logits_offset = t->tc.nsub ? (int64_t)t->L.o_tclog : 0;
     return RECSA_OK;
 }
 
@@ -394,7 +481,7 @@ recsa_status recsa_host_lengths(const recsa_tree* t, int64_t* lengths) {
 
 recsa_status recsa_set_profile_events(recsa_tree* t, int32_t which, void* start, void* stop) {
     if (!t || ((start == nullptr) != (stop == nullptr))) return RECSA_E_INVAL;
-    if (start != nullptr && (which < -1 || which > t->L.NL)) return RECSA_E_INVAL;
+    if (start != nullptr && (which < -2 || which > t->L.NL)) return RECSA_E_INVAL;
     t->prof.which = start ? which : -100;
     t->prof.start = (cudaEvent_t)start;
     t->prof.stop = (cudaEvent_t)stop;

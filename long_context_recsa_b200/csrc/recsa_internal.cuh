@@ -48,6 +48,24 @@ struct QueryView {
     int64_t pos0;
     int q_begin;               // first global query index of this wave
     int nq;                    // queries in this wave
+    // optional precomputed logits of level pre_level (tensor-core prefill path):
+    // pre[((qloc * Hkv + kvh) * G + g) * pre_stride + j], already scaled; used by a
+    // query only when pre_level is its first scored level.  nullptr: none.
+    const float* pre;
+    int pre_level;
+    int pre_stride;
+};
+
+// Buffers of the tensor-core prefill path (inside the workspace when enabled).
+struct TcView {
+    uint32_t* a_hi;            // [Hkv][MB][D/32] slice images of 128 rows x 128 B
+    uint32_t* a_lo;
+    uint32_t* b_hi;            // [Hkv][NB][D/32] slice images of 256 rows x 128 B
+    uint32_t* b_lo;
+    float* logits;             // [nsub][Hkv][G][npad]
+    int nsub;                  // queries per product
+    int npad;                  // logits row length (multiple of 256, >= C*k)
+    int MB, NB;                // M tiles (of 128 rows) and N tiles (of 256 nodes) per head
 };
 
 // Workspace carve-up.
@@ -232,7 +250,14 @@ struct ProfHook {
 
 inline void prof_mark(const ProfHook* p, int which, bool before, cudaStream_t s) {
     if (p == nullptr || p->which != which || p->start == nullptr) return;
-    cudaEventRecordWithFlags(before ? p->start : p->stop, s, cudaEventRecordExternal);
+    // inside a stream capture the record becomes an external event node of the graph
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cs);
+    cudaEvent_t ev = before ? p->start : p->stop;
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, s);
 }
 
 // ----------------------------------------------------------------------------
@@ -292,6 +317,10 @@ cudaError_t launch_append_one(const TreeView& tv, const WorkView& wv, const void
 cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
                           const void* v_new, int n, int dtype, cudaStream_t s,
                           const ProfHook* prof = nullptr);
+cudaError_t launch_prefill_top_tc(const TreeView& tv, const WorkView& wv, const QueryView& qv,
+                                  const TcView& tc, int lt, int64_t a_max, int dtype, cudaStream_t s,
+                                  const ProfHook* prof = nullptr);
+cudaError_t prepare_tc_kernels(int D);
 cudaError_t launch_select_attend(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                  int dtype, cudaStream_t s, const ProfHook* prof = nullptr);
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype);

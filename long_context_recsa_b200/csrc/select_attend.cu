@@ -824,29 +824,54 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
     // ---- the warp's parent groups and their blocks (K then V) ----
     const int P = (j1 > j0) ? cdiv(j1 - j0 + C - 1, C, lgC) : 0;
     const int nw = warp < P ? (P - warp + kWarps - 1) / kWarps : 0;
+    // logits already computed for this level (tensor-core prefill): no K blocks
+    const bool pre = !L0 && qv.pre != nullptr && level == qv.pre_level && level == lstar;
+    const int nk = pre ? 0 : nw;   // blocks [0, nk) are K, [nk, nk + nw) are V
     const WarpRing R{ring + (size_t)warp * nsw * slot_bytes, bars + warp * nsw, nsw, slot_bytes,
                      wv.status};
     auto group_first = [&](int jb) -> int64_t {
         return identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
     };
     auto issue = [&](int q) {
-        const int i = q < nw ? q : q - nw;
+        const int i = q < nk ? q : q - nk;
         const int jb = j0 + (warp + kWarps * i) * C;
-        ring_issue<T, D>(R, q, q < nw ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
+        ring_issue<T, D>(R, q, q < nk ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
     };
     if (lane == 0)
-        for (int q = 0; q < nsw && q < 2 * nw; ++q) issue(q);
+        for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
 
     // 1. scores of the chunk
-    for (int i = 0; i < nw; ++i) {
-        const unsigned char* blk = ring_wait(R, i);
-        const int jb = j0 + (warp + kWarps * i) * C;
-        const int nch = min(C, j0 + n_sc - jb);
-        if (nch > 0)
-            score_parent<T, D, G, !L0>(blk, jb, j0, nch, group_first(jb), wv.rope, p_q, rc4, qsm,
-                                       tv.scale, s, key, nodes, CH);
+    if (pre) {
+        // the query's list is [0..a_t] (identity): entry j is node j
+        const float* prow = qv.pre + (int64_t)(qloc * tv.Hkv + kvh) * G * qv.pre_stride;
+        for (int i = 0; i < nw; ++i) {
+            const int jb = j0 + (warp + kWarps * i) * C;
+            const int nch = min(C, j0 + n_sc - jb);
+            for (int c = lane; c < nch; c += 32) {
+                const int r = jb - j0 + c;
+                float imp = 0.f;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float v = __ldcg(prow + (int64_t)g * qv.pre_stride + jb + c);
+                    s[g * CH + r] = v;
+                    imp += v;
+                }
+                nodes[r] = jb + c;
+                key[r] = ordered_key(imp * (1.0f / G));
+            }
+        }
         __syncwarp();
-        if (lane == 0 && i + nsw < 2 * nw) issue(i + nsw);
+    } else {
+        for (int i = 0; i < nw; ++i) {
+            const unsigned char* blk = ring_wait(R, i);
+            const int jb = j0 + (warp + kWarps * i) * C;
+            const int nch = min(C, j0 + n_sc - jb);
+            if (nch > 0)
+                score_parent<T, D, G, !L0>(blk, jb, j0, nch, group_first(jb), wv.rope, p_q, rc4,
+                                           qsm, tv.scale, s, key, nodes, CH);
+            __syncwarp();
+            if (lane == 0 && i + nsw < nk + nw) issue(i + nsw);
+        }
     }
     for (int i = threadIdx.x; i < n_sc; i += kThreads) flag[i] = 0;
     // every warp's scores are written before any thread reads the chunk's (at
@@ -911,14 +936,14 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
 #pragma unroll
         for (int e = 0; e < V2; ++e) acc[g][e] = make_float2(0.f, 0.f);
     for (int i = 0; i < nw; ++i) {
-        const int q = nw + i;
+        const int q = nk + i;
         const unsigned char* blk = ring_wait(R, q);
         const int jb = j0 + (warp + kWarps * i) * C;
         const int nrow = min(C, j0 + n_sc - jb);
         if (nrow > 0 && fm[0] > -INFINITY)
             accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
         __syncwarp();
-        if (lane == 0 && q + nsw < 2 * nw) issue(q + nsw);
+        if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
     }
     __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
     finish_partial<T, D, G>(acc, lsum, fm, red, outp);

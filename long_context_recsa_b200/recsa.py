@@ -46,6 +46,9 @@ class RecsaTreeInfoC(ctypes.Structure):
         ("capacity", ctypes.c_int64),
         ("batch", ctypes.c_int32),
         ("max_queries", ctypes.c_int32),
+        ("tc_queries", ctypes.c_int32),
+        ("tc_row_stride", ctypes.c_int32),
+        ("tc_logits_offset", ctypes.c_int64),
     ]
 
 
@@ -192,6 +195,8 @@ class RecsaTree:
         _check(lib.recsa_tree_info(h, ctypes.byref(info)), "recsa_tree_info")
         self.n_sel_levels = info.n_sel_levels
         self.splits, self.splits0 = info.splits, info.splits0
+        self.tc_queries, self.tc_row_stride = info.tc_queries, info.tc_row_stride
+        self.tc_logits_offset = info.tc_logits_offset
 
     def __del__(self):
         h = getattr(self, "handle", None)

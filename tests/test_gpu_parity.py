@@ -207,3 +207,67 @@ def test_long_lists_sampled_select(R, k, L):
     bounded by a sampled threshold; sets must still be exact."""
     run_decode_case(R, config_id=17, B=2, Hkv=2, Hq=8, d=128, C=16, k=k, lengths=[L, L - 777],
                     dtype="bf16", cap=L, n_needles=16)
+
+
+def test_prefill_tensor_core_top_level(R):
+    """Prefill on a tree with max_queries >= 128 scores the first scored level with
+    one tensor-core product per group of rows.  The product's logits equal
+    scale * <R(a_t) q, R(j) K_j> over the stored level (fp64 here) within fp32
+    rounding, and sampled rows match the oracle: selections exact except at
+    near-ties, outputs within 2e-2."""
+    from oracle import recsa_oracle as O
+    C, k, d, Hkv, Hq = 16, 64, 128, 2, 8
+    L = 40000
+    n = 160                       # one product of 128 rows, then one of 32
+    pos0 = L - n
+    G = Hq // Hkv
+    scale = 1.0 / np.sqrt(d)
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype="bf16", pooler_w=w)
+    K, V, Q = H.make_inputs(18, 1, Hkv, Hq, d, L, [L], "bf16", q_rows=n, n_needles=16)
+    small = R.RecsaTree(cfg, L, 1, max_queries=64, k0=K, v0=V)
+    assert small.tc_queries == 0
+    del small
+    tree = R.RecsaTree(cfg, L, 1, max_queries=128, k0=K, v0=V)
+    assert tree.tc_queries == 128
+    tree.recsa_build([L])
+    Out, sel, cnt = tree.prefill(Q, pos0, with_sel=True)
+    torch.cuda.synchronize()
+    assert tree.recsa_get_status() == R.RECSA_OK
+
+    # 1. the last product's logits (rows 128..159 of the chunk) against fp64
+    lt = 2
+    assert (pos0 + n - 1) // C ** lt >= k and (pos0 + n - 1) // C ** (lt + 1) < k
+    nrows, stride = n - 128, tree.tc_row_stride
+    off = tree.tc_logits_offset
+    logits = tree.workspace[off: off + 4 * nrows * Hkv * G * stride].view(torch.float32)
+    logits = logits.reshape(nrows, Hkv, G, stride).double().cpu().numpy()
+    Kl, _ = tree.level_tables(lt)
+    worst = 0.0
+    for qi in (0, 13, nrows - 1):
+        t = pos0 + 128 + qi
+        a = t // C ** lt
+        for h in range(Hkv):
+            qg = H.to64(Q[0, 128 + qi, h * G:(h + 1) * G])
+            kr = H.to64(Kl[0, h, :a + 1])
+            ref = O.level_logits(qg, kr, a, np.arange(a + 1), scale, 1e6)
+            got = logits[qi, h, :, :a + 1]
+            bound = 1e-5 * scale * np.outer(np.linalg.norm(qg, axis=1), np.linalg.norm(kr, axis=1))
+            err = np.abs(got - ref)
+            worst = max(worst, float(np.max(err / bound)))
+            assert np.all(err <= bound), f"row {qi} head {h}: logit error {err.max()}"
+    print("tensor-core logits: worst error / bound", worst)
+
+    # 2. sampled rows of both products against the oracle
+    NL = tree.n_sel_levels
+    for h in range(Hkv):
+        levels = O.build_tree(H.to64(K[0, h, :L]), H.to64(V[0, h, :L]), C,
+                              np.asarray(w, dtype=np.float64), "bf16")
+        for i in (0, 64, 127, 128, n - 1):
+            t = pos0 + i
+            qg = H.to64(Q[0, i, h * G:(h + 1) * G])
+            res = O.select_and_attend(levels, qg, t, C, k, base=1e6)
+            cur = H.check_selection(levels, qg, t, C, k, 1e6, res, sel[i, h].cpu().numpy(),
+                                    cnt[i, h].cpu().numpy(), NL)
+            err = H.max_abs(H.to64(Out[0, i, h * G:(h + 1) * G]), cur.out)
+            assert err <= H.TOL_OUT["bf16"], f"row {i} head {h}: output max-abs {err}"
