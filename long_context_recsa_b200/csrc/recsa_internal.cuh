@@ -261,6 +261,25 @@ inline void prof_mark(const ProfHook* p, int which, bool before, cudaStream_t s)
 }
 
 // ----------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel on the stream is finishing.
+// It must pass pdl_wait() before it reads or writes any global memory that kernel
+// touches; pdl_wait() returns once that kernel has completed and its writes are
+// visible.  pdl_launch_dependents() lets the next kernel start launching.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Launch attribute that allows the overlap above.
+inline cudaLaunchAttribute pdl_attribute() {
+    cudaLaunchAttribute a = {};
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
+// ----------------------------------------------------------------------------
 // TMA bulk copies into shared memory, completed on an mbarrier (no multicast)
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -47,7 +47,7 @@ struct Shape {
 // shared-memory layout of the select/attend kernels
 // ----------------------------------------------------------------------------
 struct Smem {
-    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, samp, misc, bars, ring, red, total;
+    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, misc, bars, ring, red, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
@@ -67,8 +67,7 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
     L.flag = o;  o = align16(o + sizeof(unsigned char) * CH);
     L.par = o;   o = align16(o + sizeof(int) * k);
     L.mkey = o;  o = align16(o + sizeof(uint32_t) * NA);
-    L.hist = o;  o = align16(o + sizeof(uint32_t) * 512);
-    L.samp = o;  o = align16(o + sizeof(uint32_t) * (NA > 0 ? kThreads : 0));
+    L.hist = o;  o = align16(o + sizeof(uint32_t) * 1024);   // >= kSelBins / 2, radix 512
     L.misc = o;  o = align16(o + sizeof(int) * 64);
     L.bars = o;  o = align16(o + sizeof(uint64_t) * kWarps * 2);
     o = (o + 127) & ~size_t(127);
@@ -228,69 +227,157 @@ __device__ int block_select_ranks(const uint32_t* keys, int n, uint32_t T, int n
     return tot;
 }
 
+// Same ranks for a list of at most 16 * kThreads keys: each thread takes a run of
+// a multiple of 4 consecutive keys, read once with 16-byte loads into registers
+// (runs may read up to 15 words past n; those words are never counted).
+template <typename Fn>
+__device__ void block_select_ranks_short(const uint32_t* keys, int n, uint32_t T, int need_eq,
+                                         int cnt_eq, int lo, int hi, int* misc, Fn fn) {
+    constexpr int MAXI = 16;
+    const int ipt = (((n + kThreads - 1) / kThreads) + 3) & ~3;
+    const int i0 = threadIdx.x * ipt;
+    uint32_t kv[MAXI];
+#pragma unroll
+    for (int u = 0; u < MAXI; u += 4) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (u < ipt && i0 + u < n) w = *reinterpret_cast<const uint4*>(keys + i0 + u);
+        kv[u] = w.x; kv[u + 1] = w.y; kv[u + 2] = w.z; kv[u + 3] = w.w;
+    }
+    const bool all_eq = (cnt_eq == need_eq);
+    int tot, eq_rank = 0;
+    if (!all_eq) {
+        int ceq = 0;
+#pragma unroll
+        for (int u = 0; u < MAXI; ++u) ceq += (u < ipt && i0 + u < n && kv[u] == T);
+        eq_rank = block_excl_scan(ceq, misc + kMiscScan, tot);
+    }
+    uint32_t selm = 0;
+    int er = eq_rank;
+#pragma unroll
+    for (int u = 0; u < MAXI; ++u) {
+        if (u < ipt && i0 + u < n) {
+            bool sel = kv[u] > T;
+            if (kv[u] == T) { sel = all_eq || er < need_eq; ++er; }
+            selm |= (uint32_t)sel << u;
+        }
+    }
+    int r = block_excl_scan(__popc(selm), misc + kMiscScan, tot);
+    while (selm) {
+        const int u = __ffs(selm) - 1;
+        selm &= selm - 1;
+        const int i = i0 + u;
+        if (i >= lo && i < hi) fn(i, r);
+        ++r;
+    }
+}
+
 // Exact top-K (0 < K < M) of the M keys of mkey in list order; calls mark(j, rank)
 // for every selected list position j in [lo, hi), rank = its position among the
-// selected in list order.  A threshold T0 estimated from a 256-key sample bounds a
-// compact candidate list (keys >= T0, in list order, packed as (key, position) in
-// mkey); the exact radix select and the ranks then run on that list.  When the
-// estimate misses (fewer than K or more than kCap candidates) the whole list is
-// used.  Both paths give the same result.  mkey holds cap_words words, so the
-// compact list takes at most cap_words / 2 pairs.
+// selected in list order.  One pass histograms the leading kSelBits bits of every
+// key (two 16-bit bin counts per word); a suffix count over the bins finds the bin
+// that holds the K-th largest key.  The keys of that bin (usually about a hundred)
+// are ranked exactly against each other (key descending, position ascending); the
+// one ranked K - above - 1 is the threshold T.  The ranks in list order then follow
+// from T.  A bin larger than kSelCand keys (heavy ties) uses the radix select.
+// hist: kSelBins / 2 words.
+constexpr int kSelBits = 11;
+constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelCand = 384;
+enum { kMiscCand = 3, kMiscT = 13, kMiscNeedEq = 14, kMiscCntEq = 15 };
+
 template <typename Fn>
-__device__ void select_topk(uint32_t* mkey, int M, int K, int cap_words, uint32_t* hist,
-                            uint32_t* sample, int* misc, int lo, int hi, Fn mark) {
-    constexpr int NS = kThreads;     // sample size, one key per thread
-    constexpr int IPT = 16;          // keys per thread held in registers while compacting
-    const int kCap = min(2048, cap_words / 2);   // compact list capacity in pairs
+__device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* misc, int lo, int hi,
+                            Fn mark) {
+    constexpr int SH = 32 - kSelBits;
+    constexpr int BPT = kSelBins / kThreads;   // bins per thread
     const int tid = threadIdx.x;
-    uint32_t T;
-    int need_eq, cnt_eq, n0 = 0;
-    bool compact = false;
-    if (M > 2 * NS && M <= IPT * kThreads) {
-        sample[tid] = mkey[(int)(((int64_t)tid * M) / NS)];
-        __syncthreads();
-        int q = (int)(((int64_t)(K + (3 * K) / 5 + 32) * NS + M - 1) / M);
-        q = min(max(q, 1), NS - 1);
-        uint32_t T0;
-        int ne0, ce0;
-        block_threshold(sample, NS, q, hist, misc, T0, ne0, ce0);
-        const int i0 = tid * IPT;
-        uint32_t kr[IPT];
-        int c = 0;
-#pragma unroll
-        for (int u = 0; u < IPT; ++u) {
-            const int i = i0 + u;
-            kr[u] = i < M ? mkey[i] : 0u;
-            c += (i < M && kr[u] >= T0) ? 1 : 0;
-        }
-        int tot;
-        int off = block_excl_scan(c, misc + kMiscScan, tot);   // every load is done past its barriers
-        if (tot >= K && tot <= kCap) {
-            uint2* pairs = reinterpret_cast<uint2*>(mkey);
-#pragma unroll
-            for (int u = 0; u < IPT; ++u) {
-                const int i = i0 + u;
-                if (i < M && kr[u] >= T0) pairs[off++] = make_uint2(kr[u], (uint32_t)i);
-            }
-            __syncthreads();
-            compact = true;
-            n0 = tot;
+    for (int i = tid; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
+    if (tid == 0) misc[kMiscCand] = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < M; i0 += kThreads) {
+        const int i = i0 + tid;
+        if (i < M) {
+            const uint32_t dig = mkey[i] >> SH;
+            atomicAdd(&hist[dig >> 1], 1u << (16 * (dig & 1)));
         }
     }
-    if (compact) {
-        const uint2* pairs = reinterpret_cast<const uint2*>(mkey);
-        block_threshold(mkey, n0, K, hist, misc, T, need_eq, cnt_eq, 2);
-        block_select_ranks(
-            mkey, n0, T, need_eq, cnt_eq, 0, n0, misc,
-            [&](int ic, int r) {
-                const int j = (int)pairs[ic].y;
-                if (j >= lo && j < hi) mark(j, r);
-            },
-            2);
+    __syncthreads();
+    // thread t owns bins kSelBins-1-BPT*t-u, u = 0..BPT-1 (descending key order)
+    uint32_t cnt8[BPT];
+    int tot = 0;
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) {
+        const int bin = kSelBins - 1 - BPT * tid - u;
+        cnt8[u] = (hist[bin >> 1] >> (16 * (bin & 1))) & 0xFFFFu;
+        tot += (int)cnt8[u];
+    }
+    int all;
+    const int excl = block_excl_scan(tot, misc + kMiscScan, all);
+    if (excl < K && K <= excl + tot) {
+        int run = excl;
+#pragma unroll
+        for (int u = 0; u < BPT; ++u) {
+            if (run + (int)cnt8[u] >= K) {
+                misc[kMiscDigit] = kSelBins - 1 - BPT * tid - u;
+                misc[kMiscAbove] = run;
+                misc[kMiscCount] = (int)cnt8[u];
+                break;
+            }
+            run += (int)cnt8[u];
+        }
+    }
+    __syncthreads();
+    const uint32_t bd = (uint32_t)misc[kMiscDigit];
+    const int need = K - misc[kMiscAbove];   // keys to take from bin bd: 1..cnt
+    const int cnt = misc[kMiscCount];
+    uint32_t T;
+    int need_eq, cnt_eq;
+    if (cnt <= kSelCand) {
+        // the bin's (key, position) pairs, in any order, into the free histogram
+        uint2* cand = reinterpret_cast<uint2*>(hist);
+        for (int i = tid; i < M; i += kThreads) {
+            const uint32_t kk = mkey[i];
+            if ((kk >> SH) == bd) cand[atomicAdd(&misc[kMiscCand], 1)] = make_uint2(kk, (uint32_t)i);
+        }
+        __syncthreads();
+        for (int c = tid; c < cnt; c += kThreads) {
+            const uint2 me = cand[c];
+            int gt = 0, eq = 0, eq_before = 0;
+            int j = 0;
+            for (; j + 8 <= cnt; j += 8) {   // eight loads in flight per step
+                uint4 o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) o[u] = *reinterpret_cast<const uint4*>(cand + j + 2 * u);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    gt += (o[u].x > me.x) + (o[u].z > me.x);
+                    eq += (o[u].x == me.x) + (o[u].z == me.x);
+                    eq_before += ((o[u].x == me.x) & (o[u].y < me.y)) + ((o[u].z == me.x) & (o[u].w < me.y));
+                }
+            }
+            for (; j < cnt; ++j) {
+                const uint2 o = cand[j];
+                gt += o.x > me.x;
+                eq += o.x == me.x;
+                eq_before += (o.x == me.x) & (o.y < me.y);
+            }
+            if (gt + eq_before == need - 1) {
+                misc[kMiscT] = (int)me.x;
+                misc[kMiscNeedEq] = need - gt;
+                misc[kMiscCntEq] = eq;
+            }
+        }
+        __syncthreads();
+        T = (uint32_t)misc[kMiscT];
+        need_eq = misc[kMiscNeedEq];
+        cnt_eq = misc[kMiscCntEq];
     } else {
         block_threshold(mkey, M, K, hist, misc, T, need_eq, cnt_eq);
-        block_select_ranks(mkey, M, T, need_eq, cnt_eq, lo, hi, misc, mark);
     }
+    if (M <= 16 * kThreads)
+        block_select_ranks_short(mkey, M, T, need_eq, cnt_eq, lo, hi, misc, mark);
+    else
+        block_select_ranks(mkey, M, T, need_eq, cnt_eq, lo, hi, misc, mark);
 }
 
 // ----------------------------------------------------------------------------
@@ -395,8 +482,8 @@ __device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int
 // KG lanes by a reduce-scatter.
 // ----------------------------------------------------------------------------
 template <typename T, int D, int G, bool WITH_KEY>
-__device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, int j0, int nch,
-                                             int64_t first, const float2* rope, int p_q,
+__device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, int next_jb, int j0,
+                                             int nch, int64_t first, const float2* rope, int p_q,
                                              const float4* rc4, const float* qsm, float scale,
                                              float* s, uint32_t* key, int* nodes, int CH) {
     using S = Shape<T, D>;
@@ -409,6 +496,8 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
     const int lane = threadIdx.x & 31;
     const int c8 = lane % KG, kg = lane / KG;
     float2 qlo[G][V2], qhi[G][V2];
+    if (next_jb >= 0)   // the warp's next group: its rope row into L1 while this one runs
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(rope + (int64_t)(p_q - next_jb) * H + c8 * VEC));
     {
         const float4* qcs =
             reinterpret_cast<const float4*>(rope + (int64_t)(p_q - jb) * H + c8 * VEC);
@@ -430,34 +519,39 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
     for (int cb = 0; cb < nch; cb += KPW * U) {
         float v[NV];
 #pragma unroll
+        // branch-free over the U keys so their FMA chains interleave: a key past the
+        // group reads row 0 (always staged) and its value is never stored
         for (int u = 0; u < U; ++u) {
             const int c = cb + u * KPW + kg;
-            float2 a2[G];
+            const int cr = c < nch ? c : 0;
+            const unsigned char* row = blk + cr * kRow;
+            float2 kl[V2], kh[V2];
+            unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + c8 * 16), kl);
+            unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + H * (int)sizeof(T) + c8 * 16), kh);
+            const float4* rc = rc4 + cr * (H / 2) + c8;
+            float2 alo[G], ahi[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) a2[g] = make_float2(0.f, 0.f);
-            if (c < nch) {
-                const unsigned char* row = blk + c * kRow;
-                float2 kl[V2], kh[V2];
-                unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + c8 * 16), kl);
-                unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + H * (int)sizeof(T) + c8 * 16), kh);
-                const float4* rc = rc4 + (c * H + c8 * VEC) / 2;
+            for (int g = 0; g < G; ++g) {
+                alo[g] = make_float2(0.f, 0.f);
+                ahi[g] = make_float2(0.f, 0.f);
+            }
 #pragma unroll
-                for (int w = 0; w < V2; ++w) {
-                    const float4 cs = rc[w];   // (cos v, cos v+1, sin v, sin v+1) of c * theta
-                    const float2 co = make_float2(cs.x, cs.y);
-                    const float2 si = make_float2(cs.z, cs.w);
-                    const float2 ns = __fmul2_rn(si, make_float2(-1.f, -1.f));
-                    const float2 ka = __ffma2_rn(kh[w], ns, __fmul2_rn(kl[w], co));
-                    const float2 kb = __ffma2_rn(kl[w], si, __fmul2_rn(kh[w], co));
+            for (int w = 0; w < V2; ++w) {
+                const float4 cs = rc[w * KG];   // (cos v, cos v+1, sin v, sin v+1) of c * theta
+                const float2 co = make_float2(cs.x, cs.y);
+                const float2 si = make_float2(cs.z, cs.w);
+                const float2 ns = make_float2(-cs.z, -cs.w);
+                const float2 ka = __ffma2_rn(kh[w], ns, __fmul2_rn(kl[w], co));
+                const float2 kb = __ffma2_rn(kl[w], si, __fmul2_rn(kh[w], co));
 #pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        a2[g] = __ffma2_rn(qlo[g][w], ka, a2[g]);
-                        a2[g] = __ffma2_rn(qhi[g][w], kb, a2[g]);
-                    }
+                for (int g = 0; g < G; ++g) {
+                    alo[g] = __ffma2_rn(qlo[g][w], ka, alo[g]);
+                    ahi[g] = __ffma2_rn(qhi[g][w], kb, ahi[g]);
                 }
             }
 #pragma unroll
-            for (int g = 0; g < G; ++g) v[u * G + g] = a2[g].x + a2[g].y;
+            for (int g = 0; g < G; ++g)
+                v[u * G + g] = (alo[g].x + ahi[g].x) + (alo[g].y + ahi[g].y);
         }
         if constexpr (RS) {
             reduce_scatter<NV, KG>(v, c8);
@@ -501,16 +595,20 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
     }
 }
 
-// Unrotated query heads of one KV head (fp32) and the C child rotations R(c)
-// (cos, sin, -sin) into shared memory.
+// Unrotated query heads of one KV head (fp32) and the C child rotations R(c) into
+// shared memory.  R(c) is stored per pair couple (v, v+1) as (cos v, cos v+1,
+// sin v, sin v+1); couple w of the lane that owns couples [V2*c8, V2*c8 + V2) sits
+// at c * (D/4) + w * KG + c8, so the KG lanes of one key read consecutive words.
 template <typename T, int D, int G>
 __device__ __forceinline__ void stage_query(const T* qrow, const float2* rope, int C, float* qsm,
                                             float4* rc4) {
+    using S = Shape<T, D>;
+    constexpr int V2 = S::VEC / 2;
     for (int i = threadIdx.x; i < G * D; i += kThreads) qsm[i] = (float)qrow[i];
-    // R(c), c < C, as (cos v, cos v+1, sin v, sin v+1) for pair couples (v, v+1)
     for (int i = threadIdx.x; i < C * (D / 4); i += kThreads) {
+        const int c = i / (D / 4), f = i % (D / 4);
         const float2 a = rope[2 * i], bb = rope[2 * i + 1];
-        rc4[i] = make_float4(a.x, bb.x, a.y, bb.y);
+        rc4[c * (D / 4) + (f % V2) * S::KG + f / V2] = make_float4(a.x, bb.x, a.y, bb.y);
     }
 }
 
@@ -718,7 +816,6 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
     int* par = reinterpret_cast<int*>(smem + SL.par);
     uint32_t* mkey = reinterpret_cast<uint32_t*>(smem + SL.mkey);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + SL.hist);
-    uint32_t* samp = reinterpret_cast<uint32_t*>(smem + SL.samp);
     int* misc = reinterpret_cast<int*>(smem + SL.misc);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bars);
     unsigned char* ring = smem + SL.ring;
@@ -731,17 +828,18 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
     const int qloc = unit / tv.Hkv, kvh = unit % tv.Hkv;
     const int gq = qv.q_begin + qloc;
     const int b = gq / qv.n_per_b;
-    const int64_t len = wv.lens[b];
-    // loads that depend only on the unit are issued together: query heads, child
-    // rotations, and the parent list S^(level+1) when there is one
+    // inputs no earlier kernel of the step writes: the query heads and the child
+    // rotations (staged while the previous kernel may still be finishing)
     const T* qrow = reinterpret_cast<const T*>(qv.q) + ((int64_t)gq * tv.Hq + kvh * G) * D;
     stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
-    if (L0 ? NL >= 1 : level < NL) {
+    if (threadIdx.x < kWarps * nsw) mbar_init(&bars[threadIdx.x], 1);
+    mbar_fence_init();
+    pdl_wait();
+    const int64_t len = wv.lens[b];
+    if (L0 ? NL >= 1 : level < NL) {   // the parent list S^(level+1)
         const int32_t* src = wv.sel + ((int64_t)unit * NL + level) * k;
         for (int i = threadIdx.x; i < k; i += kThreads) par[i] = src[i];
     }
-    if (threadIdx.x < kWarps * nsw) mbar_init(&bars[threadIdx.x], 1);
-    mbar_fence_init();
     const int64_t t = (qv.mode == 0) ? len - 1 : qv.pos0 + (gq - b * qv.n_per_b);
     const bool valid = t >= 0 && t < len;
     const int lstar = valid ? first_scored_level(t, C, lgC, k) : 0;
@@ -837,6 +935,12 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
         const int jb = j0 + (warp + kWarps * i) * C;
         ring_issue<T, D>(R, q, q < nk ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
     };
+    if (identity && rs == D && threadIdx.x == 0 && j1 > j0) {
+        // the first scored level was not prefetched by a level above: its chunk
+        // (contiguous rows j0..j1) goes to L2 ahead of the ring
+        prefetch_l2(kbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
+        prefetch_l2(vbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
+    }
     if (lane == 0)
         for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
 
@@ -866,9 +970,10 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
             const unsigned char* blk = ring_wait(R, i);
             const int jb = j0 + (warp + kWarps * i) * C;
             const int nch = min(C, j0 + n_sc - jb);
+            const int next_jb = (i + 1 < nw) ? jb + kWarps * C : -1;
             if (nch > 0)
-                score_parent<T, D, G, !L0>(blk, jb, j0, nch, group_first(jb), wv.rope, p_q, rc4,
-                                           qsm, tv.scale, s, key, nodes, CH);
+                score_parent<T, D, G, !L0>(blk, jb, next_jb, j0, nch, group_first(jb), wv.rope, p_q,
+                                           rc4, qsm, tv.scale, s, key, nodes, CH);
             __syncwarp();
             if (lane == 0 && i + nsw < nk + nw) issue(i + nsw);
         }
@@ -889,6 +994,7 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
             const int lo = r * chunk, hi = min(M, lo + chunk);
             if (hi <= lo) break;
             const uint32_t* rk = cluster.map_shared_rank(key, r);
+#pragma unroll 4
             for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
         }
         cluster_arrive();   // remote reads done; matched by cluster_wait() before exit
@@ -908,7 +1014,7 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
             nrs = D;
         }
         if (K1 > 0)   // k = 1: only the current node is selected
-            select_topk(mkey, M, K1, NA, hist, samp, misc, j0, j0 + n_sc, [&](int i, int r) {
+            select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, [&](int i, int r) {
                 const int node = nodes[i - j0];
                 sel_ws[r] = node;
                 if (sel_usr) sel_usr[r] = node;
@@ -1018,23 +1124,32 @@ static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, co
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = sm;
         cfg.stream = s;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)wv.SPL;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1] = pdl_attribute();
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         prof_mark(prof, level, true, s);
         cudaError_t e =
             cudaLaunchKernelEx(&cfg, level_kernel<T, D, G, false>, tv, wv, qv, level, CH, NA, nsw);
         prof_mark(prof, level, false, s);
         if (e != cudaSuccess) return e;
     }
+    cudaLaunchConfig_t cfg0 = {};
+    cfg0.gridDim = dim3((unsigned)wv.NS0, units, 1);
+    cfg0.blockDim = dim3(kThreads, 1, 1);
+    cfg0.dynamicSmemBytes = sm0;
+    cfg0.stream = s;
+    cudaLaunchAttribute attr0[1] = {pdl_attribute()};
+    cfg0.attrs = attr0;
+    cfg0.numAttrs = 1;
     prof_mark(prof, 0, true, s);
-    level_kernel<T, D, G, true><<<dim3((unsigned)wv.NS0, units), kThreads, sm0, s>>>(tv, wv, qv, 0,
-                                                                                    CH0, 0, nsw);
+    cudaError_t e0 = cudaLaunchKernelEx(&cfg0, level_kernel<T, D, G, true>, tv, wv, qv, 0, CH0, 0, nsw);
     prof_mark(prof, 0, false, s);
+    if (e0 != cudaSuccess) return e0;
     return cudaGetLastError();
 }
 

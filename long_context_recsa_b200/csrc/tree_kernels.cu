@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(256) append_one_kernel(TreeView tv, WorkView w
     const int nwarps = blockDim.x >> 5;
     const int off = lane * N;
     for (int i = threadIdx.x; i < C * C; i += blockDim.x) alpha[i] = wv.alpha[i];
+    pdl_wait();
     const int64_t t = wv.lens[b];
     __syncthreads();
     if (t + 1 > tv.cap) {
@@ -456,10 +457,20 @@ template <typename T, int D>
 static cudaError_t append_one_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
                                    const void* v_new, cudaStream_t s, const ProfHook* prof) {
     const size_t sm = sizeof(double) * 2 * D * (size_t)(tv.n_levels > 1 ? tv.n_levels - 1 : 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tv.B * tv.Hkv), 1, 1);
+    cfg.blockDim = dim3(kAppendThreads, 1, 1);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1] = {pdl_attribute()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     prof_mark(prof, -1, true, s);
-    append_one_kernel<T, D><<<tv.B * tv.Hkv, kAppendThreads, sm, s>>>(
-        tv, wv, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new));
+    cudaError_t e = cudaLaunchKernelEx(&cfg, append_one_kernel<T, D>, tv, wv,
+                                       reinterpret_cast<const T*>(k_new),
+                                       reinterpret_cast<const T*>(v_new));
     prof_mark(prof, -1, false, s);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
