@@ -1032,6 +1032,8 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
         __syncthreads();
     }
 
+    // the next kernel may start launching: what remains here is this CTA's partial
+    pdl_launch_dependents();
     // 4. softmax partial over the unselected (level) or all (level 0) entries
     float lsum[G];
     // (scratch: the histogram area; the ring, and so red, still holds V blocks)
