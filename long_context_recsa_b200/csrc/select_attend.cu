@@ -37,10 +37,47 @@ namespace recsa {
 template <typename T, int D>
 struct Shape {
     static constexpr int VEC = VecOf<T>::N;   // elements per 16-byte load
-    static constexpr int KG = D / (2 * VEC);  // lanes per key (each lane: VEC rotary pairs)
-    static constexpr int KPW = 32 / KG;       // keys per warp step
+    // scoring: LPK lanes per key, each owning PPL consecutive rotary pairs (CPL
+    // couples of two pairs) of the low and of the high half of the key
+    static constexpr int LPK = 16;
+    static constexpr int PPL = D / 2 / LPK;
+    static constexpr int CPL = PPL / 2;
+    static constexpr int KPW = 32 / LPK;      // keys per warp step
     static constexpr int RPL = D / VEC;       // lanes per value row
     static constexpr int RPW = 32 / RPL;      // value rows per warp step
+};
+
+// PPL consecutive elements (a multiple of 2) as CPL fp32 pairs.
+template <typename T, int PPL>
+struct PairLoad;
+template <>
+struct PairLoad<__nv_bfloat16, 4> {
+    static __device__ __forceinline__ void get(const unsigned char* p, float2 (&o)[2]) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p);
+        o[0] = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+        o[1] = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+    }
+};
+template <>
+struct PairLoad<__nv_bfloat16, 2> {
+    static __device__ __forceinline__ void get(const unsigned char* p, float2 (&o)[1]) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        o[0] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+};
+template <>
+struct PairLoad<float, 4> {
+    static __device__ __forceinline__ void get(const unsigned char* p, float2 (&o)[2]) {
+        const float4 w = *reinterpret_cast<const float4*>(p);
+        o[0] = make_float2(w.x, w.y);
+        o[1] = make_float2(w.z, w.w);
+    }
+};
+template <>
+struct PairLoad<float, 2> {
+    static __device__ __forceinline__ void get(const unsigned char* p, float2 (&o)[1]) {
+        o[0] = *reinterpret_cast<const float2*>(p);
+    }
 };
 
 // ----------------------------------------------------------------------------
@@ -478,8 +515,10 @@ __device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int
 // Scores of one parent group staged in shared memory: row c of blk is the key of
 // list entry jb + c (c < nch).  s[g][r] = scale * <R(p_q - jb) q_g, R(c) K>, the
 // order-preserving key of the mean over heads, and the node index first + c,
-// at r = jb - j0 + c.  Packed fp32x2 arithmetic; each key is reduced over its
-// KG lanes by a reduce-scatter.
+// at r = jb - j0 + c.  LPK lanes share a key, each rotating and multiplying its
+// PPL pairs of both halves with packed fp32x2 arithmetic; the U keys of a lane
+// are computed branch-free so their chains interleave, and the partial dot
+// products are combined by a reduce-scatter over the LPK lanes.
 // ----------------------------------------------------------------------------
 template <typename T, int D, int G, bool WITH_KEY>
 __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, int next_jb, int j0,
@@ -487,30 +526,32 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
                                              const float4* rc4, const float* qsm, float scale,
                                              float* s, uint32_t* key, int* nodes, int CH) {
     using S = Shape<T, D>;
-    constexpr int VEC = S::VEC, KG = S::KG, KPW = S::KPW, H = D / 2, V2 = VEC / 2;
+    constexpr int LPK = S::LPK, PPL = S::PPL, CPL = S::CPL, KPW = S::KPW, H = D / 2;
     constexpr int kRow = D * (int)sizeof(T);
+    constexpr int kHalf = H * (int)sizeof(T);
     constexpr int U = 4;                       // keys per lane per batch
-    constexpr int NV = U * G;                  // values reduced over a key group
-    constexpr int R = NV / KG;                 // values per lane after reduce-scatter
-    constexpr bool RS = (NV % KG == 0) && (R >= 1) && (G % (R > 0 ? R : 1) == 0);
+    constexpr int NV = U * G;                  // values reduced over a key's lanes
+    constexpr int R = NV / LPK;                // values per lane after reduce-scatter
+    constexpr bool RS = (NV % LPK == 0) && (R >= 1) && (G % (R > 0 ? R : 1) == 0);
     const int lane = threadIdx.x & 31;
-    const int c8 = lane % KG, kg = lane / KG;
-    float2 qlo[G][V2], qhi[G][V2];
+    const int cl = lane % LPK, kg = lane / LPK;
+    const int off = cl * PPL * (int)sizeof(T);   // byte offset of the lane's pairs in a half
+    // the query heads rotated by R(p_q - jb), the lane's couples only
+    float2 qlo[G][CPL], qhi[G][CPL];
     if (next_jb >= 0)   // the warp's next group: its rope row into L1 while this one runs
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(rope + (int64_t)(p_q - next_jb) * H + c8 * VEC));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(rope + (int64_t)(p_q - next_jb) * H + cl * PPL));
     {
-        const float4* qcs =
-            reinterpret_cast<const float4*>(rope + (int64_t)(p_q - jb) * H + c8 * VEC);
+        const float4* qcs = reinterpret_cast<const float4*>(rope + (int64_t)(p_q - jb) * H + cl * PPL);
 #pragma unroll
-        for (int w = 0; w < V2; ++w) {
+        for (int w = 0; w < CPL; ++w) {
             const float4 cs = __ldg(qcs + w);   // (cos v, sin v, cos v+1, sin v+1)
             const float2 co = make_float2(cs.x, cs.z);
             const float2 si = make_float2(cs.y, cs.w);
             const float2 ns = make_float2(-cs.y, -cs.w);
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float2 x1 = *reinterpret_cast<const float2*>(qsm + g * D + c8 * VEC + 2 * w);
-                const float2 x2 = *reinterpret_cast<const float2*>(qsm + g * D + H + c8 * VEC + 2 * w);
+                const float2 x1 = *reinterpret_cast<const float2*>(qsm + g * D + cl * PPL + 2 * w);
+                const float2 x2 = *reinterpret_cast<const float2*>(qsm + g * D + H + cl * PPL + 2 * w);
                 qlo[g][w] = __ffma2_rn(x2, ns, __fmul2_rn(x1, co));
                 qhi[g][w] = __ffma2_rn(x1, si, __fmul2_rn(x2, co));
             }
@@ -518,17 +559,16 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
     }
     for (int cb = 0; cb < nch; cb += KPW * U) {
         float v[NV];
+        // a key past the group reads row 0 (always staged); its value is never stored
 #pragma unroll
-        // branch-free over the U keys so their FMA chains interleave: a key past the
-        // group reads row 0 (always staged) and its value is never stored
         for (int u = 0; u < U; ++u) {
             const int c = cb + u * KPW + kg;
             const int cr = c < nch ? c : 0;
             const unsigned char* row = blk + cr * kRow;
-            float2 kl[V2], kh[V2];
-            unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + c8 * 16), kl);
-            unpack_pairs<T>(*reinterpret_cast<const uint4*>(row + H * (int)sizeof(T) + c8 * 16), kh);
-            const float4* rc = rc4 + cr * (H / 2) + c8;
+            float2 kl[CPL], kh[CPL];
+            PairLoad<T, PPL>::get(row + off, kl);
+            PairLoad<T, PPL>::get(row + kHalf + off, kh);
+            const float4* rc = rc4 + cr * (H / 2) + cl;
             float2 alo[G], ahi[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -536,8 +576,8 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
                 ahi[g] = make_float2(0.f, 0.f);
             }
 #pragma unroll
-            for (int w = 0; w < V2; ++w) {
-                const float4 cs = rc[w * KG];   // (cos v, cos v+1, sin v, sin v+1) of c * theta
+            for (int w = 0; w < CPL; ++w) {
+                const float4 cs = rc[w * LPK];   // (cos v, cos v+1, sin v, sin v+1) of c * theta
                 const float2 co = make_float2(cs.x, cs.y);
                 const float2 si = make_float2(cs.z, cs.w);
                 const float2 ns = make_float2(-cs.z, -cs.w);
@@ -554,8 +594,8 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
                 v[u * G + g] = (alo[g].x + ahi[g].x) + (alo[g].y + ahi[g].y);
         }
         if constexpr (RS) {
-            reduce_scatter<NV, KG>(v, c8);
-            const int u = (c8 * R) / G, g0 = (c8 * R) % G;
+            reduce_scatter<NV, LPK>(v, cl);
+            const int u = (cl * R) / G, g0 = (cl * R) % G;
             const int c = cb + u * KPW + kg;
             float imp = 0.f;
 #pragma unroll
@@ -575,11 +615,11 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
 #pragma unroll
             for (int i = 0; i < NV; ++i)
 #pragma unroll
-                for (int o = 1; o < KG; o <<= 1) v[i] += __shfl_xor_sync(kFull, v[i], o);
+                for (int o = 1; o < LPK; o <<= 1) v[i] += __shfl_xor_sync(kFull, v[i], o);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int c = cb + u * KPW + kg;
-                if (c < nch && c8 == 0) {
+                if (c < nch && cl == 0) {
                     const int r = jb - j0 + c;
                     float imp = 0.f;
 #pragma unroll
@@ -597,18 +637,18 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
 
 // Unrotated query heads of one KV head (fp32) and the C child rotations R(c) into
 // shared memory.  R(c) is stored per pair couple (v, v+1) as (cos v, cos v+1,
-// sin v, sin v+1); couple w of the lane that owns couples [V2*c8, V2*c8 + V2) sits
-// at c * (D/4) + w * KG + c8, so the KG lanes of one key read consecutive words.
+// sin v, sin v+1); couple w of the lane that owns couples [CPL*l, CPL*l + CPL)
+// sits at c * (D/4) + w * LPK + l, so the LPK lanes of one key read consecutive
+// 16-byte words.
 template <typename T, int D, int G>
 __device__ __forceinline__ void stage_query(const T* qrow, const float2* rope, int C, float* qsm,
                                             float4* rc4) {
     using S = Shape<T, D>;
-    constexpr int V2 = S::VEC / 2;
     for (int i = threadIdx.x; i < G * D; i += kThreads) qsm[i] = (float)qrow[i];
     for (int i = threadIdx.x; i < C * (D / 4); i += kThreads) {
         const int c = i / (D / 4), f = i % (D / 4);
         const float2 a = rope[2 * i], bb = rope[2 * i + 1];
-        rc4[c * (D / 4) + (f % V2) * S::KG + f / V2] = make_float4(a.x, bb.x, a.y, bb.y);
+        rc4[c * (D / 4) + (f % S::CPL) * S::LPK + f / S::CPL] = make_float4(a.x, bb.x, a.y, bb.y);
     }
 }
 
