@@ -371,10 +371,27 @@ __device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* m
     int need_eq, cnt_eq;
     if (cnt <= kSelCand) {
         // the bin's (key, position) pairs, in any order, into the free histogram
+        // two passes without atomics: each warp counts the bin's keys in its slice of
+        // the list, then writes them after the counts of the warps before it
         uint2* cand = reinterpret_cast<uint2*>(hist);
-        for (int i = tid; i < M; i += kThreads) {
-            const uint32_t kk = mkey[i];
-            if ((kk >> SH) == bd) cand[atomicAdd(&misc[kMiscCand], 1)] = make_uint2(kk, (uint32_t)i);
+        const int lane = tid & 31, warp = tid >> 5;
+        const int per = (((M + kWarps - 1) / kWarps) + 31) & ~31;
+        const int w0 = warp * per, w1 = min(M, w0 + per);
+        int wcnt = 0;
+        for (int i = w0 + lane; i - lane < w1; i += 32) {
+            const bool in = i < w1 && (mkey[i] >> SH) == bd;
+            wcnt += __popc(__ballot_sync(kFull, in));
+        }
+        if (lane == 0) misc[kMiscScan + warp] = wcnt;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; ++w) base += misc[kMiscScan + w];
+        for (int i = w0 + lane; i - lane < w1; i += 32) {
+            const uint32_t kk = i < w1 ? mkey[i] : 0u;
+            const bool in = i < w1 && (kk >> SH) == bd;
+            const unsigned bal = __ballot_sync(kFull, in);
+            if (in) cand[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(kk, (uint32_t)i);
+            base += __popc(bal);
         }
         __syncthreads();
         for (int c = tid; c < cnt; c += kThreads) {
@@ -696,7 +713,9 @@ __device__ __forceinline__ void softmax_weights(float* s, int n, const unsigned 
 }
 
 // o_g += p_g * V for the rows of one staged parent group: row c of blk is the
-// value of entry jb + c (c < nrow), skipped when flagged (selected).
+// value of entry jb + c (c < nrow), left out when flagged (selected).  Branch-free
+// so the unrolled rows pipeline their loads: a row past the group reads row 0 and,
+// like a flagged row, gets weight 0.
 template <typename T, int D, int G>
 __device__ __forceinline__ void accum_parent(const unsigned char* blk, int jb, int j0, int nrow,
                                              const unsigned char* flag, const float* s, int CH,
@@ -708,20 +727,19 @@ __device__ __forceinline__ void accum_parent(const unsigned char* blk, int jb, i
     const int c = lane % S::RPL, rr = lane / S::RPL;
 #pragma unroll 4
     for (int cb = 0; cb < nrow; cb += S::RPW) {
-        const int cr = cb + rr;
-        if (cr < nrow) {
-            const int r = jb - j0 + cr;
-            if (!flag || flag[r] == 0) {
-                float2 v[V2];
-                unpack_pairs<T>(*reinterpret_cast<const uint4*>(blk + cr * kRow + c * 16), v);
+        const int cr0 = cb + rr;
+        const bool in_group = cr0 < nrow;
+        const int cr = in_group ? cr0 : 0;
+        const int r = jb - j0 + cr;
+        const bool inc = in_group && (!flag || flag[r] == 0);
+        float2 v[V2];
+        unpack_pairs<T>(*reinterpret_cast<const uint4*>(blk + cr * kRow + c * 16), v);
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float p = s[g * CH + r];
-                    const float2 p2 = make_float2(p, p);
+        for (int g = 0; g < G; ++g) {
+            const float p = inc ? s[g * CH + r] : 0.f;
+            const float2 p2 = make_float2(p, p);
 #pragma unroll
-                    for (int e = 0; e < V2; ++e) acc[g][e] = __ffma2_rn(p2, v[e], acc[g][e]);
-                }
-            }
+            for (int e = 0; e < V2; ++e) acc[g][e] = __ffma2_rn(p2, v[e], acc[g][e]);
         }
     }
 }
@@ -1059,8 +1077,6 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
                 sel_ws[r] = node;
                 if (sel_usr) sel_usr[r] = node;
                 flag[i - j0] = 1;
-                // the children of a selected node are the next level's rows
-                prefetch_children<T, D>(nk, nv, nrs, (int64_t)C * node, C);
             });
         if (crank == 0 && threadIdx.x == 0) {
             const int64_t cur = apow(t, level, C, lgC);
@@ -1070,6 +1086,10 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
                                     (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1));
         }
         __syncthreads();
+        // the children of this chunk's selected nodes are the next level's rows: to L2,
+        // each thread for its own entries, so the requests go out in parallel
+        for (int i = threadIdx.x; i < n_sc; i += kThreads)
+            if (flag[i]) prefetch_children<T, D>(nk, nv, nrs, (int64_t)C * nodes[i], C);
     }
 
     // the next kernel may start launching: what remains here is this CTA's partial
