@@ -130,8 +130,15 @@ RECSA_API recsa_status recsa_build(recsa_tree* tree, const int64_t* lengths, voi
  * by append(n) is bitwise equal to build(L+n)), and L grows by n.  If L + n would
  * exceed capacity the sequence is left unchanged and the status word records
  * RECSA_E_CAPACITY (the host also rejects this synchronously while its own copy
- * of the lengths is current, i.e. outside graph replays).  With n == 1 the whole
- * update (new rows, every ancestor, the length) is one kernel launch. */
+ * of the lengths is current, i.e. outside graph replays).
+ * With n == 1 this call writes the new rows and the lengths only (one launch).  The
+ * re-pooling of the new tokens' ancestors is carried out by the next call on the
+ * handle: recsa_decode does it inside its level-0 launch (a decode at the new
+ * position reads none of those ancestors: each is the current node of its level,
+ * never scored and never a summary); every other call (recsa_append,
+ * recsa_prefill_chunk, recsa_get_status) first runs it as a separate launch on its
+ * own stream, and recsa_build makes it unnecessary.  A caller that reads the level
+ * tables directly does so after one of those calls. */
 RECSA_API recsa_status recsa_append(recsa_tree* tree, const void* k_new, const void* v_new, int32_t n,
                           void* stream);
 

@@ -194,7 +194,19 @@ struct recsa_tree {
     int64_t host_len[RECSA_MAX_BATCH];
     ProfHook prof;
     TcView tc;                 // tensor-core prefill buffers (tc.nsub == 0: none)
+    // a single-token append left the ancestors of the new tokens to re-pool: the next
+    // decode does it in its level-0 launch, any other call first
+    bool walk_pending;
 };
+
+// Runs a pending ancestor re-pooling on `stream` (before a call that needs the
+// complete tree).
+static recsa_status finish_walk(recsa_tree* t, cudaStream_t stream) {
+    if (!t->walk_pending) return RECSA_OK;
+    t->walk_pending = false;
+    return launch_append_walk(t->tv, t->wv, t->cfg.dtype, stream) == cudaSuccess ? RECSA_OK
+                                                                                 : RECSA_E_CUDA;
+}
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -320,6 +332,7 @@ recsa_status recsa_build(recsa_tree* t, const int64_t* lengths, void* stream) {
     if (!t || !lengths) return RECSA_E_INVAL;
     for (int b = 0; b < t->B; ++b)
         if (lengths[b] < 0 || lengths[b] > t->cap) return RECSA_E_CAPACITY;
+    t->walk_pending = false;   // the build pools every node anew
     cudaError_t e = launch_build(t->tv, t->wv, lengths, t->cfg.dtype, (cudaStream_t)stream);
     if (e != cudaSuccess) return RECSA_E_CUDA;
     for (int b = 0; b < t->B; ++b) t->host_len[b] = lengths[b];
@@ -333,9 +346,11 @@ recsa_status recsa_append(recsa_tree* t, const void* k_new, const void* v_new, i
     for (int b = 0; b < t->B; ++b)
         if (t->host_len[b] + n > t->cap) return RECSA_E_CAPACITY;
     const cudaStream_t s = (cudaStream_t)stream;
+    if (finish_walk(t, s) != RECSA_OK) return RECSA_E_CUDA;
     cudaError_t e;
     if (n == 1) {
-        e = launch_append_one(t->tv, t->wv, k_new, v_new, t->cfg.dtype, s, &t->prof);
+        e = launch_append_token(t->tv, t->wv, k_new, v_new, t->cfg.dtype, s, &t->prof);
+        if (e == cudaSuccess) t->walk_pending = true;
     } else {
         e = launch_append(t->tv, t->wv, k_new, v_new, n, t->cfg.dtype, s, &t->prof);
     }
@@ -358,9 +373,12 @@ recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_
     qv.pos0 = 0;
     qv.q_begin = 0;
     qv.nq = t->B;
+    qv.walk = t->walk_pending ? 1 : 0;
     cudaError_t e =
         launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof);
-    return e == cudaSuccess ? RECSA_OK : RECSA_E_CUDA;
+    if (e != cudaSuccess) return RECSA_E_CUDA;
+    t->walk_pending = false;
+    return RECSA_OK;
 }
 
 // t / C^l and the first scored level of position t (host side of Eq.3's sizes).
@@ -385,6 +403,7 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
     for (int b = 0; b < t->B; ++b)
         if (pos0 + n > t->host_len[b]) return RECSA_E_CAPACITY;
     const cudaStream_t s = (cudaStream_t)stream;
+    if (finish_walk(t, s) != RECSA_OK) return RECSA_E_CUDA;
     auto base_view = [&]() {
         QueryView qv = {};
         qv.q = Q;
@@ -435,6 +454,7 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
 
 recsa_status recsa_get_status(recsa_tree* t, void* stream) {
     if (!t) return RECSA_E_INVAL;
+    if (finish_walk(t, (cudaStream_t)stream) != RECSA_OK) return RECSA_E_CUDA;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RECSA_E_CUDA;
     uint32_t v = 0;
     if (cudaMemcpy(&v, t->wv.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)

@@ -54,6 +54,9 @@ struct QueryView {
     const float* pre;
     int pre_level;
     int pre_stride;
+    // decode only: the level-0 launch also re-pools the ancestors of each sequence's
+    // newest token (extra CTAs after the attention CTAs)
+    int walk;
 };
 
 // Buffers of the tensor-core prefill path (inside the workspace when enabled).
@@ -330,9 +333,10 @@ cudaError_t launch_init_workspace(const TreeView& tv, const WorkView& wv, double
                                   cudaStream_t s);
 cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* lengths,
                          int dtype, cudaStream_t s);
-cudaError_t launch_append_one(const TreeView& tv, const WorkView& wv, const void* k_new,
-                              const void* v_new, int dtype, cudaStream_t s,
-                              const ProfHook* prof = nullptr);
+cudaError_t launch_append_token(const TreeView& tv, const WorkView& wv, const void* k_new,
+                                const void* v_new, int dtype, cudaStream_t s,
+                                const ProfHook* prof = nullptr);
+cudaError_t launch_append_walk(const TreeView& tv, const WorkView& wv, int dtype, cudaStream_t s);
 cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
                           const void* v_new, int n, int dtype, cudaStream_t s,
                           const ProfHook* prof = nullptr);

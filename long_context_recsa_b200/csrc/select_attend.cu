@@ -28,7 +28,7 @@
 // fixed rotations R(0..C-1), staged in shared memory.
 #include <cooperative_groups.h>
 
-#include "recsa_internal.cuh"
+#include "pool.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -858,6 +858,24 @@ template <typename T, int D, int G, bool L0>
 __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkView wv, QueryView qv,
                                                             int level, int CH, int NA, int nsw) {
     extern __shared__ __align__(128) unsigned char smem[];
+    if constexpr (L0) {
+        // CTAs past the attention grid re-pool the ancestors of each sequence's newest
+        // token (one CTA per sequence and KV head); nothing here reads them
+        const int units = qv.nq * tv.Hkv;
+        if ((int)blockIdx.y >= units) {
+            const int ci = ((int)blockIdx.y - units) * (int)gridDim.x + (int)blockIdx.x;
+            if (ci >= tv.B * tv.Hkv) return;
+            double* alpha = reinterpret_cast<double*>(smem);
+            double* pre = alpha + RECSA_MAX_C * RECSA_MAX_C;
+            for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
+            pdl_wait();
+            const int b = ci / tv.Hkv, h = ci % tv.Hkv;
+            const int64_t t = wv.lens[b] - 1;
+            __syncthreads();
+            if (t >= 1) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha);
+            return;
+        }
+    }
     constexpr int kRow = D * (int)sizeof(T);
     constexpr int V2 = VecOf<T>::N / 2;
     const int k = tv.k, C = tv.C, lgC = tv.lgC, K1 = k - 1, NL = wv.NL;
@@ -1167,8 +1185,10 @@ static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
     }
+    const size_t walk = ancestor_walk_smem(kMaxLevels, D);
     return cudaFuncSetAttribute(level_kernel<T, D, G, true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm0);
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(sm0 > walk ? sm0 : walk));
 }
 
 template <typename T, int D, int G>
@@ -1201,9 +1221,13 @@ static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, co
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg0 = {};
-    cfg0.gridDim = dim3((unsigned)wv.NS0, units, 1);
+    // with a pending ancestor walk, extra rows of CTAs (one CTA per sequence and KV head)
+    const unsigned walk_rows =
+        qv.walk ? (unsigned)((tv.B * tv.Hkv + wv.NS0 - 1) / wv.NS0) : 0u;
+    const size_t walk_sm = ancestor_walk_smem(tv.n_levels, D);
+    cfg0.gridDim = dim3((unsigned)wv.NS0, units + walk_rows, 1);
     cfg0.blockDim = dim3(kThreads, 1, 1);
-    cfg0.dynamicSmemBytes = sm0;
+    cfg0.dynamicSmemBytes = (qv.walk && walk_sm > sm0) ? walk_sm : sm0;
     cfg0.stream = s;
     cudaLaunchAttribute attr0[1] = {pdl_attribute()};
     cfg0.attrs = attr0;

@@ -9,160 +9,13 @@
 // K), and are rounded once to the storage dtype; the next level pools the rounded
 // values.  Build and append perform the same operations in the same order, so an
 // appended tree is bitwise equal to a rebuilt one.
-#include "recsa_internal.cuh"
+#include "pool.cuh"
 
 namespace recsa {
-
-// Lanes own D/32 consecutive dimensions, so one warp instruction reads a whole
-// row and every dimension is summed by one lane in child order.
-template <typename T, int D>
-struct PoolShape {
-    static constexpr int DPL = D / 32;   // dimensions per lane
-};
-
-// DPL consecutive elements as floats (exact widening), and back.
-template <typename T, int N>
-struct Dims;
-template <>
-struct Dims<float, 4> {
-    static __device__ __forceinline__ void load(const float* p, float (&x)[4]) {
-        const float4 v = *reinterpret_cast<const float4*>(p);
-        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-    }
-    static __device__ __forceinline__ void store(float* p, const float (&x)[4]) {
-        *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
-    }
-};
-template <>
-struct Dims<float, 2> {
-    static __device__ __forceinline__ void load(const float* p, float (&x)[2]) {
-        const float2 v = *reinterpret_cast<const float2*>(p);
-        x[0] = v.x; x[1] = v.y;
-    }
-    static __device__ __forceinline__ void store(float* p, const float (&x)[2]) {
-        *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
-    }
-};
-template <>
-struct Dims<__nv_bfloat16, 4> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[4]) {
-        const uint2 v = *reinterpret_cast<const uint2*>(p);
-        x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xffff0000u);
-        x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xffff0000u);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&x)[4]) {
-        uint2 v;
-        v.x = (__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xffff0000u);
-        v.y = (__float_as_uint(x[2]) >> 16) | (__float_as_uint(x[3]) & 0xffff0000u);
-        *reinterpret_cast<uint2*>(p) = v;
-    }
-};
-template <>
-struct Dims<__nv_bfloat16, 2> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[2]) {
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
-        x[0] = __uint_as_float(v << 16); x[1] = __uint_as_float(v & 0xffff0000u);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&x)[2]) {
-        *reinterpret_cast<uint32_t*>(p) =
-            (__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xffff0000u);
-    }
-};
-
-// softmax(w[0..m-1]) for every m = 1..C, fp64, into alpha[(m-1)*C + c].
-__device__ void fill_alpha(const float* w, int C, double* alpha) {
-    for (int idx = threadIdx.x; idx < C * C; idx += blockDim.x) {
-        int m = idx / C + 1, c = idx % C;
-        double v = 0.0;
-        if (c < m) {
-            double mx = (double)w[0];
-            for (int j = 1; j < m; ++j) mx = fmax(mx, (double)w[j]);
-            double sum = 0.0;
-            for (int j = 0; j < m; ++j) sum += exp((double)w[j] - mx);
-            v = exp((double)w[c] - mx) / sum;
-        }
-        alpha[idx] = v;
-    }
-}
-
-// Adds children rows [r_lo, r_hi) (row stride rs elements) of one parent to this
-// lane's fp64 sums, in child order: ak += alpha_m[r] * K_r (fused), av += V_r.
-// Rows are loaded B at a time ahead of the arithmetic.
-template <typename T, int D, int B = 8>
-__device__ __forceinline__ void pool_rows(const T* sk, const T* sv, int64_t rs, int r_lo, int r_hi,
-                                          const double* alpha_m, double (&ak)[D / 32],
-                                          double (&av)[D / 32]) {
-    constexpr int N = PoolShape<T, D>::DPL;
-    const int off = (threadIdx.x & 31) * N;
-    for (int r0 = r_lo; r0 < r_hi; r0 += B) {
-        float kx[B][N], vx[B][N];
-#pragma unroll
-        for (int u = 0; u < B; ++u)
-            if (r0 + u < r_hi) {
-                Dims<T, N>::load(sk + (r0 + u) * rs + off, kx[u]);
-                Dims<T, N>::load(sv + (r0 + u) * rs + off, vx[u]);
-            }
-#pragma unroll
-        for (int u = 0; u < B; ++u)
-            if (r0 + u < r_hi) {
-                const double al = alpha_m[r0 + u];
-#pragma unroll
-                for (int e = 0; e < N; ++e) {
-                    ak[e] = fma(al, (double)kx[u][e], ak[e]);
-                    av[e] += (double)vx[u][e];
-                }
-            }
-    }
-}
-
-// Rounds one parent's sums to storage: K = ak, V = av / m.  Returns the stored
-// values widened to float in (fk, fv).
-template <typename T, int D>
-__device__ __forceinline__ void pool_store(const double (&ak)[D / 32], const double (&av)[D / 32],
-                                           int m, T* dk, T* dv, float (&fk)[D / 32],
-                                           float (&fv)[D / 32]) {
-    constexpr int N = PoolShape<T, D>::DPL;
-    const int off = (threadIdx.x & 31) * N;
-    const double dm = (double)m;
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-        fk[e] = (float)store_round<T>(ak[e]);
-        fv[e] = (float)store_round<T>(av[e] / dm);
-    }
-    Dims<T, N>::store(dk + off, fk);
-    Dims<T, N>::store(dv + off, fv);
-}
-
-// One warp pools the m children of one parent (the whole node).
-template <typename T, int D>
-__device__ __forceinline__ void warp_pool_node(const T* sk, const T* sv, int64_t rs, int m,
-                                               const double* alpha_m, T* dk, T* dv) {
-    constexpr int N = PoolShape<T, D>::DPL;
-    double ak[N], av[N];
-#pragma unroll
-    for (int e = 0; e < N; ++e) { ak[e] = 0.0; av[e] = 0.0; }
-    pool_rows<T, D>(sk, sv, rs, 0, m, alpha_m, ak, av);
-    float fk[N], fv[N];
-    pool_store<T, D>(ak, av, m, dk, dv, fk, fv);
-}
 
 __device__ __forceinline__ int64_t ceil_div_pow(int64_t n, int C, int l) {
     for (int i = 0; i < l; ++i) n = (n + C - 1) / C;
     return n;
-}
-
-template <typename T>
-__device__ __forceinline__ void level_rows(const TreeView& tv, int l, int b, int h, const T*& k,
-                                           const T*& v, int64_t& rs) {
-    if (l == 0) {
-        k = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + h * tv.s_h);
-        v = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + h * tv.s_h);
-        rs = tv.s_t;
-    } else {
-        k = level_k<T>(tv, l, b, h);
-        v = level_v<T>(tv, l, b, h);
-        rs = tv.D;
-    }
 }
 
 // ----------------------------------------------------------------------------
@@ -304,90 +157,33 @@ __global__ void commit_lengths_kernel(WorkView wv, int B, int64_t add, int64_t c
 }
 
 // ----------------------------------------------------------------------------
-// single-token append: one CTA per (sequence, KV head), one launch per step.
-// Token t = L is written at level 0; its ancestor at level l is node t / C^l, whose
-// m = (t / C^(l-1)) mod C + 1 children are m-1 complete nodes and, last, the
-// ancestor at level l-1.  Warps first sum the complete children of every level in
-// parallel (fp64, child order, kept in shared memory); warp 0 then walks the levels
-// bottom-up adding the one new term per level, so the serial part is a few fused
-// multiply-adds per level.  The last CTA of a sequence advances its length.
+// single-token append, split in two:
+//   append_token_kernel writes token t = L of every (sequence, KV head) at level 0
+//     and advances the length (the last CTA of a sequence does);
+//   the ancestors of t are re-pooled by ancestor_walk, either in extra CTAs of the
+//     next decode's level-0 kernel or by append_walk_kernel.  A decode at t reads no
+//     ancestor of t: each is the current node of its level, never scored and never
+//     a summary, and every other node it lists is complete.
 // ----------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(256) append_one_kernel(TreeView tv, WorkView wv, const T* knew,
-                                                         const T* vnew) {
-    extern __shared__ double pre[];   // [levels][2][D]: K then V sums of complete children
-    __shared__ double alpha[RECSA_MAX_C * RECSA_MAX_C];
-    constexpr int N = PoolShape<T, D>::DPL;
+__global__ void __launch_bounds__(64) append_token_kernel(TreeView tv, WorkView wv, const T* knew,
+                                                          const T* vnew) {
     constexpr int VEC = VecOf<T>::N;
     const int bh = blockIdx.x;
     const int b = bh / tv.Hkv, h = bh % tv.Hkv;
-    const int C = tv.C, lgC = tv.lgC;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
-    const int off = lane * N;
-    for (int i = threadIdx.x; i < C * C; i += blockDim.x) alpha[i] = wv.alpha[i];
     pdl_wait();
     const int64_t t = wv.lens[b];
-    __syncthreads();
     if (t + 1 > tv.cap) {
         if (h == 0 && threadIdx.x == 0) set_status(wv.status, kStatusCapacity);
         return;
     }
+    T* k0 = reinterpret_cast<T*>(tv.k0w) + (b * tv.s_b + h * tv.s_h + t * tv.s_t);
+    T* v0 = reinterpret_cast<T*>(tv.v0w) + (b * tv.s_b + h * tv.s_h + t * tv.s_t);
     const T* kn = knew + (int64_t)bh * D;
     const T* vn = vnew + (int64_t)bh * D;
-    // levels 1..nl are pooled: level l exists while level l-1 has more than one node
-    int nl = 0;
-    for (int64_t x = t; x >= 1 && nl + 1 < tv.n_levels; x = cdiv64(x, C, lgC)) ++nl;
-    // the new level-0 row is copied by the last warp, which has no level of its own
-    // unless there are more levels than warps, so its loads overlap the others'
-    if (warp == nwarps - 1) {
-        T* k0 = reinterpret_cast<T*>(tv.k0w) + (b * tv.s_b + h * tv.s_h + t * tv.s_t);
-        T* v0 = reinterpret_cast<T*>(tv.v0w) + (b * tv.s_b + h * tv.s_h + t * tv.s_t);
-        for (int e = lane; e < D / VEC; e += 32) {
-            *reinterpret_cast<uint4*>(k0 + e * VEC) = *reinterpret_cast<const uint4*>(kn + e * VEC);
-            *reinterpret_cast<uint4*>(v0 + e * VEC) = *reinterpret_cast<const uint4*>(vn + e * VEC);
-        }
-    }
-
-    for (int l = 1 + warp; l <= nl; l += nwarps) {
-        int64_t x = t;   // ancestor index at level l-1
-        for (int j = 1; j < l; ++j) x = cdiv64(x, C, lgC);
-        const int64_t i = cdiv64(x, C, lgC);
-        const int m = (int)(x - i * C) + 1;
-        const T *sk, *sv;
-        int64_t rs;
-        level_rows<T>(tv, l - 1, b, h, sk, sv, rs);
-        double ak[N], av[N];
-#pragma unroll
-        for (int e = 0; e < N; ++e) { ak[e] = 0.0; av[e] = 0.0; }
-        pool_rows<T, D, 16>(sk + i * C * rs, sv + i * C * rs, rs, 0, m - 1, alpha + (m - 1) * C,
-                            ak, av);
-#pragma unroll
-        for (int e = 0; e < N; ++e) {
-            pre[(2 * (l - 1)) * D + off + e] = ak[e];
-            pre[(2 * (l - 1) + 1) * D + off + e] = av[e];
-        }
-    }
-    __syncthreads();
-    if (warp == 0) {
-        float ck[N], cv[N];   // the newest child: the token, then each new ancestor
-        Dims<T, N>::load(kn + off, ck);
-        Dims<T, N>::load(vn + off, cv);
-        int64_t x = t;
-        for (int l = 1; l <= nl; ++l) {
-            const int64_t i = cdiv64(x, C, lgC);
-            const int m = (int)(x - i * C) + 1;
-            const double al = alpha[(m - 1) * C + (m - 1)];
-            double ak[N], av[N];
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-                ak[e] = fma(al, (double)ck[e], pre[(2 * (l - 1)) * D + off + e]);
-                av[e] = pre[(2 * (l - 1) + 1) * D + off + e] + (double)cv[e];
-            }
-            pool_store<T, D>(ak, av, m, level_k<T>(tv, l, b, h) + i * D,
-                             level_v<T>(tv, l, b, h) + i * D, ck, cv);
-            x = i;
-        }
+    for (int e = threadIdx.x; e < D / VEC; e += blockDim.x) {
+        *reinterpret_cast<uint4*>(k0 + e * VEC) = *reinterpret_cast<const uint4*>(kn + e * VEC);
+        *reinterpret_cast<uint4*>(v0 + e * VEC) = *reinterpret_cast<const uint4*>(vn + e * VEC);
     }
     // every CTA of sequence b has read lens[b] before it counts itself here
     __syncthreads();
@@ -398,6 +194,22 @@ __global__ void __launch_bounds__(256) append_one_kernel(TreeView tv, WorkView w
             wv.lens[b] = t + 1;
         }
     }
+}
+
+// The ancestors of each sequence's newest token t = L - 1, one CTA per (sequence,
+// KV head).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) append_walk_kernel(TreeView tv, WorkView wv) {
+    extern __shared__ double walk_smem[];
+    double* alpha = walk_smem;
+    double* pre = walk_smem + RECSA_MAX_C * RECSA_MAX_C;
+    const int b = blockIdx.x / tv.Hkv, h = blockIdx.x % tv.Hkv;
+    for (int i = threadIdx.x; i < tv.C * tv.C; i += blockDim.x) alpha[i] = wv.alpha[i];
+    pdl_wait();
+    const int64_t t = wv.lens[b] - 1;
+    __syncthreads();
+    if (t < 1) return;
+    ancestor_walk<T, D>(tv, b, h, t, pre, alpha);
 }
 
 // ----------------------------------------------------------------------------
@@ -449,27 +261,36 @@ static cudaError_t append_impl(const TreeView& tv, const WorkView& wv, const voi
     return cudaGetLastError();
 }
 
-constexpr int kAppendThreads = 256;
-
-static size_t append_one_smem(int D) { return sizeof(double) * 2 * D * (kMaxLevels - 1); }
-
 template <typename T, int D>
-static cudaError_t append_one_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
-                                   const void* v_new, cudaStream_t s, const ProfHook* prof) {
-    const size_t sm = sizeof(double) * 2 * D * (size_t)(tv.n_levels > 1 ? tv.n_levels - 1 : 1);
+static cudaError_t append_token_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
+                                     const void* v_new, cudaStream_t s, const ProfHook* prof) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tv.B * tv.Hkv), 1, 1);
-    cfg.blockDim = dim3(kAppendThreads, 1, 1);
-    cfg.dynamicSmemBytes = sm;
+    cfg.blockDim = dim3(64, 1, 1);
     cfg.stream = s;
     cudaLaunchAttribute attr[1] = {pdl_attribute()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     prof_mark(prof, -1, true, s);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, append_one_kernel<T, D>, tv, wv,
+    cudaError_t e = cudaLaunchKernelEx(&cfg, append_token_kernel<T, D>, tv, wv,
                                        reinterpret_cast<const T*>(k_new),
                                        reinterpret_cast<const T*>(v_new));
     prof_mark(prof, -1, false, s);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t append_walk_impl(const TreeView& tv, const WorkView& wv, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tv.B * tv.Hkv), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = ancestor_walk_smem(tv.n_levels, D);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1] = {pdl_attribute()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, append_walk_kernel<T, D>, tv, wv);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -485,8 +306,8 @@ static cudaError_t append_one_impl(const TreeView& tv, const WorkView& wv, const
 
 template <typename T, int D>
 static cudaError_t prepare_tree_impl(const TreeView&) {
-    return cudaFuncSetAttribute(append_one_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)append_one_smem(D));
+    return cudaFuncSetAttribute(append_walk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)ancestor_walk_smem(kMaxLevels, D));
 }
 
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype) {
@@ -505,9 +326,13 @@ cudaError_t launch_build(const TreeView& tv, const WorkView& wv, const int64_t* 
     RECSA_DISPATCH_TD(dtype, tv.D, build_impl, tv, wv, lengths, s);
 }
 
-cudaError_t launch_append_one(const TreeView& tv, const WorkView& wv, const void* k_new,
-                              const void* v_new, int dtype, cudaStream_t s, const ProfHook* prof) {
-    RECSA_DISPATCH_TD(dtype, tv.D, append_one_impl, tv, wv, k_new, v_new, s, prof);
+cudaError_t launch_append_token(const TreeView& tv, const WorkView& wv, const void* k_new,
+                                const void* v_new, int dtype, cudaStream_t s, const ProfHook* prof) {
+    RECSA_DISPATCH_TD(dtype, tv.D, append_token_impl, tv, wv, k_new, v_new, s, prof);
+}
+
+cudaError_t launch_append_walk(const TreeView& tv, const WorkView& wv, int dtype, cudaStream_t s) {
+    RECSA_DISPATCH_TD(dtype, tv.D, append_walk_impl, tv, wv, s);
 }
 
 cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,

@@ -271,3 +271,47 @@ def test_prefill_tensor_core_top_level(R):
                                     cnt[i, h].cpu().numpy(), NL)
             err = H.max_abs(H.to64(Out[0, i, h * G:(h + 1) * G]), cur.out)
             assert err <= H.TOL_OUT["bf16"], f"row {i} head {h}: output max-abs {err}"
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_single_appends_without_decode_equal_build(R, dtype):
+    """Single-token appends leave the ancestors to the next call: back-to-back
+    appends and a status query complete them as a separate launch, a decode inside
+    its level-0 launch.  Tables and outputs equal a fresh build bit for bit."""
+    C, k, d, Hkv, Hq, B = 16, 8, 64, 2, 4, 2
+    L0, cap = 3000, 3100
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype=dtype, pooler_w=w)
+    K, V, q = H.make_inputs(19, B, Hkv, Hq, d, cap, [cap] * B, dtype)
+    q = q[:, 0].contiguous()
+    Ka, Va = K.clone(), V.clone()
+    Ka[:, :, L0:] = 0
+    Va[:, :, L0:] = 0
+    inc = R.RecsaTree(cfg, cap, B, k0=Ka, v0=Va)
+    inc.recsa_build([L0] * B)
+
+    def tables_equal(n):
+        ref = R.RecsaTree(cfg, cap, B, k0=K.clone(), v0=V.clone())
+        ref.recsa_build([n] * B)
+        for l in range(1, ref.n_levels):
+            rows = -(-n // C ** l)
+            Ki, Vi = inc.level_tables(l)
+            Kr, Vr = ref.level_tables(l)
+            assert torch.equal(Ki[:, :, :rows], Kr[:, :, :rows]), f"K level {l} at {n}"
+            assert torch.equal(Vi[:, :, :rows], Vr[:, :, :rows]), f"V level {l} at {n}"
+        return ref
+
+    n = L0
+    for _ in range(5):
+        inc.recsa_append(K[:, :, n:n + 1].contiguous(), V[:, :, n:n + 1].contiguous())
+        n += 1
+    assert inc.recsa_get_status() == R.RECSA_OK        # completes the last append
+    tables_equal(n)
+    for _ in range(3):
+        inc.recsa_append(K[:, :, n:n + 1].contiguous(), V[:, :, n:n + 1].contiguous())
+        n += 1
+    out = inc.decode(q)[0]                              # completes it in its own launch
+    torch.cuda.synchronize()
+    ref = tables_equal(n)
+    assert torch.equal(out, ref.decode(q)[0])
+    assert inc.recsa_get_status() == R.RECSA_OK
