@@ -32,10 +32,11 @@ METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
 # ncu capture at batch 1 (profiles/level_kernels_decode524k_b1.md); a launch covers
 # batch x 8 independent units, so the batch-B figure is B times this.  Valid only
 # for the kernel sources it was taken from: any edit to them turns it into null.
-TRAFFIC_LEVEL1_B1 = {"bytes": 33_760_256 + 768,
+TRAFFIC_LEVEL1_B1 = {"bytes": 33_696_768 + 768,
                      "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
-                                 "long_context_recsa_b200/csrc/recsa_internal.cuh"],
-                     "sha256": "205cddb9d634061dab3e189d15fb56466644d673033cf909e4118b25db02ea3c"}
+                                 "long_context_recsa_b200/csrc/recsa_internal.cuh",
+                                 "long_context_recsa_b200/csrc/pool.cuh"],
+                     "sha256": "6097bdea1e6b5080d3675c9c800bcf7587188a87301373798545b15f22399bc7"}
 
 
 def captured_traffic(kernel: str, batch: int):
