@@ -83,7 +83,11 @@ extern "C" RECSA_API recsa_status recsa_decode_noalloc(
         qv.n_per_b = 1;
         qv.q_begin = 0;
         qv.nq = batch;
-        e = launch_select_attend(tv, wv, qv, cfg->dtype, s);
+        // tensor maps of the caller's tables, encoded on the host for this call
+        static thread_local KVMaps maps[kMaxLevels];
+        const bool mapped = uses_kv_maps(cfg->dtype, tv.D, cfg->C) &&
+                            encode_kv_maps(tv, maps) == cudaSuccess;
+        e = launch_select_attend(tv, wv, qv, cfg->dtype, s, nullptr, mapped ? maps : nullptr);
     }
     return e == cudaSuccess ? RECSA_OK : RECSA_E_CUDA;
 }

@@ -3,6 +3,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "recsa_internal.cuh"
 
 namespace recsa {
@@ -194,6 +196,8 @@ struct recsa_tree {
     int64_t host_len[RECSA_MAX_BATCH];
     ProfHook prof;
     TcView tc;                 // tensor-core prefill buffers (tc.nsub == 0: none)
+    KVMaps maps[kMaxLevels];   // swizzled TMA maps of every level (bf16, d = 128 trees)
+    bool has_maps;
     // a single-token append left the ancestors of the new tokens to re-pool: the next
     // decode does it in its level-0 launch, any other call first
     bool walk_pending;
@@ -319,6 +323,9 @@ recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t 
     cudaError_t e = prepare_kernels(cfg->dtype, L.D, L.G, L.SPL, L.NS0, cfg->C, cfg->k);
     if (e == cudaSuccess) e = prepare_tree_kernels(tv, cfg->dtype);
     if (e == cudaSuccess && L.tc_nsub > 0) e = prepare_tc_kernels(L.D);
+    // tables the tensor maps cannot describe (strides off 16 bytes) keep plain copies
+    t->has_maps = e == cudaSuccess && uses_kv_maps(cfg->dtype, L.D, cfg->C) &&
+                  encode_kv_maps(tv, t->maps) == cudaSuccess;
     if (e == cudaSuccess) e = launch_init_workspace(tv, wv, cfg->rope_base, (cudaStream_t)stream);
     if (e != cudaSuccess) {
         free(t);
@@ -375,7 +382,8 @@ recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_
     qv.nq = t->B;
     qv.walk = t->walk_pending ? 1 : 0;
     cudaError_t e =
-        launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof);
+        launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof,
+                             t->has_maps ? t->maps : nullptr);
     if (e != cudaSuccess) return RECSA_E_CUDA;
     t->walk_pending = false;
     return RECSA_OK;
@@ -435,7 +443,8 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
                     qv.pre_level = lt;
                     qv.pre_stride = t->tc.npad;
                 }
-                cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof);
+                cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof,
+                                                     t->has_maps ? t->maps : nullptr);
                 if (e != cudaSuccess) return RECSA_E_CUDA;
             }
         }
@@ -446,7 +455,8 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
         QueryView qv = base_view();
         qv.q_begin = q0;
         qv.nq = total - q0 < t->Qmax ? total - q0 : t->Qmax;
-        cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof);
+        cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof,
+                                                     t->has_maps ? t->maps : nullptr);
         if (e != cudaSuccess) return RECSA_E_CUDA;
     }
     return RECSA_OK;
@@ -515,3 +525,69 @@ recsa_status recsa_tree_free(recsa_tree* t) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// TMA tensor maps of the level tables (see KVMaps)
+// ----------------------------------------------------------------------------
+namespace recsa {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// One table: rows of 128 bf16 at row pitch `row_b` bytes, heads `head_b`, sequences
+// `seq_b` apart; boxes of 64 dims x C rows.
+static cudaError_t encode_table(CUtensorMap* m, const void* base, int64_t rows, int Hkv, int B,
+                                int64_t row_b, int64_t head_b, int64_t seq_b, int C) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    if (rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;   // row coordinates are int32
+    const cuuint64_t dims[4] = {128, (cuuint64_t)rows, (cuuint64_t)Hkv, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)row_b, (cuuint64_t)head_b, (cuuint64_t)seq_b};
+    const cuuint32_t box[4] = {64, (cuuint32_t)C, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t encode_kv_maps(const TreeView& tv, KVMaps* maps) {
+    for (int l = 0; l < tv.n_levels && l < kMaxLevels; ++l) {
+        cudaError_t e;
+        if (l == 0) {
+            const int64_t es = 2;
+            e = encode_table(&maps[0].k, tv.k0, tv.cap, tv.Hkv, tv.B, tv.s_t * es, tv.s_h * es,
+                             tv.s_b * es, tv.C);
+            if (e == cudaSuccess)
+                e = encode_table(&maps[0].v, tv.v0, tv.cap, tv.Hkv, tv.B, tv.s_t * es,
+                                 tv.s_h * es, tv.s_b * es, tv.C);
+        } else {
+            const int64_t rows = tv.rows[l], row_b = 256;
+            e = encode_table(&maps[l].k, tv.levels + tv.off_k[l], rows, tv.Hkv, tv.B, row_b,
+                             rows * row_b, rows * row_b * tv.Hkv, tv.C);
+            if (e == cudaSuccess)
+                e = encode_table(&maps[l].v, tv.levels + tv.off_v[l], rows, tv.Hkv, tv.B, row_b,
+                                 rows * row_b, rows * row_b * tv.Hkv, tv.C);
+        }
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace recsa

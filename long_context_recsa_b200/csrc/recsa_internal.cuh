@@ -1,6 +1,7 @@
 // Internal declarations shared by the RecSA CUDA translation units (sm_100a).
 #pragma once
 
+#include <cuda.h>   // CUtensorMap only; maps are encoded through the runtime's driver entry point
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -15,7 +16,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr unsigned kFull = 0xffffffffu;
 
 // Device status word values (first error wins).
-enum : uint32_t { kStatusOk = 0, kStatusBadQuery = 1, kStatusCapacity = 2, kStatusTimeout = 3 };
+enum : uint32_t { kStatusOk = 0, kStatusBadQuery = 1, kStatusCapacity = 2, kStatusTimeout = 3,
+                  kStatusLayout = 4 /* a staging buffer was misaligned */ };
 
 // Location of the tree in device memory.
 struct TreeView {
@@ -57,6 +59,14 @@ struct QueryView {
     // decode only: the level-0 launch also re-pools the ancestors of each sequence's
     // newest token (extra CTAs after the attention CTAs)
     int walk;
+};
+
+// TMA tensor maps of one level's K and V tables (bf16, d = 128): 4-d (d, row, KV
+// head, sequence), box 64 dims x C rows, 128-byte swizzle.  A parent group is staged
+// as two boxes (dims 0-63, 64-127) into [half][C rows][128 B] of a 1024-byte-aligned
+// slot, so 8 consecutive rows fall in 8 different swizzle phases.
+struct KVMaps {
+    CUtensorMap k, v;
 };
 
 // Buffers of the tensor-core prefill path (inside the workspace when enabled).
@@ -345,7 +355,15 @@ cudaError_t launch_prefill_top_tc(const TreeView& tv, const WorkView& wv, const 
                                   const ProfHook* prof = nullptr);
 cudaError_t prepare_tc_kernels(int D);
 cudaError_t launch_select_attend(const TreeView& tv, const WorkView& wv, const QueryView& qv,
-                                 int dtype, cudaStream_t s, const ProfHook* prof = nullptr);
+                                 int dtype, cudaStream_t s, const ProfHook* prof = nullptr,
+                                 const KVMaps* maps = nullptr);
+// Whether a tree stages its rows through swizzled tensor maps: bf16, d = 128, and
+// parent groups of a multiple of 16 rows (whole tensor-core steps).
+inline bool uses_kv_maps(int dtype, int D, int C) {
+    return dtype == RECSA_BF16 && D == 128 && C % 16 == 0 && C <= 256;
+}
+// Encodes maps[l] for levels 0 .. tv.n_levels - 1 (level 0: the caller's cache).
+cudaError_t encode_kv_maps(const TreeView& tv, KVMaps* maps);
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype);
 cudaError_t launch_set_lengths(const WorkView& wv, const int64_t* lengths, int B, cudaStream_t s);
 recsa_status views_for(const recsa_config* cfg, int64_t cap, int B, int Qmax, const void* k0,

@@ -80,6 +80,21 @@ struct PairLoad<float, 2> {
     }
 };
 
+// Rows of bf16 keys and values with d = 128 can be staged by TMA tensor copies
+// with 128-byte swizzle (the SW kernels): a parent group of C rows (C a multiple of
+// 16) fills its slot as [half][C rows][128 B], half 0 holding dims 0-63 and half 1
+// dims 64-127, and the 16-byte chunk j of row r stored at chunk j ^ (r mod 8).  The
+// rows of an 8-row tile then fall in 8 different bank groups for ldmatrix.
+template <typename T, int D>
+constexpr bool kSwzCapable = false;
+template <>
+constexpr bool kSwzCapable<__nv_bfloat16, 128> = true;
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of half `half` of row `row` in a slot.
+__device__ __forceinline__ uint32_t swz_off(int half, int row, int chunk, int C) {
+    return (uint32_t)(half * C * 128 + row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
 // ----------------------------------------------------------------------------
 // shared-memory layout of the select/attend kernels
 // ----------------------------------------------------------------------------
@@ -107,7 +122,7 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
     L.hist = o;  o = align16(o + sizeof(uint32_t) * 1024);   // >= kSelBins / 2, radix 512
     L.misc = o;  o = align16(o + sizeof(int) * 64);
     L.bars = o;  o = align16(o + sizeof(uint64_t) * kWarps * 2);
-    o = (o + 127) & ~size_t(127);
+    o = (o + 1023) & ~size_t(1023);   // swizzled slots need 1024-byte alignment
     L.ring = o;
     L.red = o;
     const size_t red_bytes = sizeof(float) * kWarps * G * (D + 1);
@@ -521,6 +536,24 @@ __device__ __forceinline__ void ring_issue(const WarpRing& R, int q, const T* ba
     }
 }
 
+// Issue block q from a tensor map: the C rows from `first` of KV head h of sequence
+// b as two swizzled boxes (dims 0-63 and 64-127).  Rows past the table arrive as
+// zeros; the full box is always delivered.  One lane.
+__device__ __forceinline__ void ring_issue_map(const WarpRing& R, int q, const CUtensorMap* map,
+                                               int64_t first, int h, int b, int C) {
+    const int s = q % R.nsw;
+    unsigned char* dst = R.slots + (size_t)s * R.slot_bytes;
+    mbar_expect_tx(&R.bars[s], (uint32_t)C * 256u);
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+        asm volatile(
+            "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+            "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst + half * C * 128)),
+            "l"(reinterpret_cast<uint64_t>(map)), "r"(half * 64), "r"((int)first), "r"(h), "r"(b),
+            "r"(smem_u32(&R.bars[s]))
+            : "memory");
+}
+
 // Wait (bounded) for block q; all lanes of the warp.
 __device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int q) {
     const int s = q % R.nsw;
@@ -537,9 +570,10 @@ __device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int
 // are computed branch-free so their chains interleave, and the partial dot
 // products are combined by a reduce-scatter over the LPK lanes.
 // ----------------------------------------------------------------------------
-template <typename T, int D, int G, bool WITH_KEY>
-__device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, int next_jb, int j0,
-                                             int nch, int64_t first, const float2* rope, int p_q,
+template <typename T, int D, int G, bool WITH_KEY, bool SW>
+__device__ __forceinline__ void score_parent(const unsigned char* blk, int C, int jb, int next_jb,
+                                             int j0, int nch, int64_t first, const float2* rope,
+                                             int p_q,
                                              const float4* rc4, const float* qsm, float scale,
                                              float* s, uint32_t* key, int* nodes, int CH) {
     using S = Shape<T, D>;
@@ -581,10 +615,17 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int jb, i
         for (int u = 0; u < U; ++u) {
             const int c = cb + u * KPW + kg;
             const int cr = c < nch ? c : 0;
-            const unsigned char* row = blk + cr * kRow;
             float2 kl[CPL], kh[CPL];
-            PairLoad<T, PPL>::get(row + off, kl);
-            PairLoad<T, PPL>::get(row + kHalf + off, kh);
+            if constexpr (SW) {
+                // the lane's 8 bytes: half of 16-byte chunk cl / 2 of each half row
+                const uint32_t in = (uint32_t)(cl & 1) * 8u;
+                PairLoad<T, PPL>::get(blk + swz_off(0, cr, cl >> 1, C) + in, kl);
+                PairLoad<T, PPL>::get(blk + swz_off(1, cr, cl >> 1, C) + in, kh);
+            } else {
+                const unsigned char* row = blk + cr * kRow;
+                PairLoad<T, PPL>::get(row + off, kl);
+                PairLoad<T, PPL>::get(row + kHalf + off, kh);
+            }
             const float4* rc = rc4 + cr * (H / 2) + cl;
             float2 alo[G], ahi[G];
 #pragma unroll
@@ -744,6 +785,31 @@ __device__ __forceinline__ void accum_parent(const unsigned char* blk, int jb, i
     }
 }
 
+// Second half of a partial: each warp has written its o rows to red[warp][g][0..D);
+// its l partials go to red[warp][g][D], then the warps are summed into the record
+// [G][D+2] = (o, m, l).
+template <int D, int G>
+__device__ __forceinline__ void partial_tail(float* lsum, const float* fm, float* red, float* outp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lsum[g] += __shfl_xor_sync(kFull, lsum[g], o);
+    if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) red[(warp * G + g) * (D + 1) + D] = lsum[g];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * (D + 1); i += kThreads) {
+        float sum = 0.f;
+        for (int w = 0; w < kWarps; ++w) sum += red[w * G * (D + 1) + i];
+        const int g = i / (D + 1), d = i % (D + 1);
+        if (d < D) outp[g * (D + 2) + d] = sum;
+        else outp[g * (D + 2) + D + 1] = sum;
+    }
+    if (threadIdx.x < G) outp[threadIdx.x * (D + 2) + D] = fm[threadIdx.x];
+}
+
 // Cross-lane and cross-warp reduction of the value accumulators and l partials
 // into the partial record [G][D+2] = (o, m, l).  red must be free.
 template <typename T, int D, int G>
@@ -762,10 +828,6 @@ __device__ __forceinline__ void finish_partial(float2 (&acc)[G][VecOf<T>::N / 2]
                 acc[g][e].x += __shfl_xor_sync(kFull, acc[g][e].x, o);
                 acc[g][e].y += __shfl_xor_sync(kFull, acc[g][e].y, o);
             }
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) lsum[g] += __shfl_xor_sync(kFull, lsum[g], o);
     if (rr == 0) {
 #pragma unroll
         for (int g = 0; g < G; ++g)
@@ -775,19 +837,122 @@ __device__ __forceinline__ void finish_partial(float2 (&acc)[G][VecOf<T>::N / 2]
                 red[(warp * G + g) * (D + 1) + c * VEC + 2 * e + 1] = acc[g][e].y;
             }
     }
-    if (lane == 0) {
+    partial_tail<D, G>(lsum, fm, red, outp);
+}
+
+// ---- value accumulation on the tensor cores (SW kernels: bf16, d = 128) ----
+// o^T[d][g] += sum_r V[r][d] p_g[r] as mma.sync m16n8k16 products with fp32
+// accumulation: M = the D value dims (D/16 tiles), N = 8 query-head columns (G used,
+// the rest zero), K = 16 rows of the group per step.  A = V^T comes straight from
+// the swizzled slot by ldmatrix.trans; B = the weights, split into a bf16 high part
+// and a bf16 remainder so that together they carry 16 significant bits (two
+// products), which keeps the accumulated output as close to an fp32 product as the
+// scalar path's.  acc[mt][0..3] holds (dim mt*16 + lane/4, heads 2*(lane%4), +1)
+// and (dim + 8, same heads).
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// The weights of rows k0 + 2t, +1 (b0) and k0 + 2t + 8, +9 (b1) for head lane/4 as
+// bf16 high parts and remainders; zero for rows past nrow, flagged rows, and head
+// columns >= G.
+template <int G>
+__device__ __forceinline__ void weight_frags(const float* s, const unsigned char* flag, int CH,
+                                             int rb, int k0, int nrow, uint32_t (&bh)[2],
+                                             uint32_t (&bl)[2]) {
+    const int lane = threadIdx.x & 31;
+    const int gi = lane >> 2, tg = lane & 3;
+    bh[0] = bh[1] = bl[0] = bl[1] = 0u;
+    if (gi < G) {
+        float p[4];
 #pragma unroll
-        for (int g = 0; g < G; ++g) red[(warp * G + g) * (D + 1) + D] = lsum[g];
+        for (int i = 0; i < 4; ++i) {
+            const int c = k0 + 2 * tg + (i & 1) + (i >> 1) * 8;
+            const int r = rb + c;
+            const bool inc = c < nrow && (!flag || flag[r] == 0);
+            p[i] = inc ? s[gi * CH + r] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(p[2 * j], p[2 * j + 1]);
+            const float2 hf = __bfloat1622float2(h);
+            bh[j] = *reinterpret_cast<const uint32_t*>(&h);
+            bl[j] = pack_bf16x2(p[2 * j] - hf.x, p[2 * j + 1] - hf.y);
+        }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < G * (D + 1); i += kThreads) {
-        float sum = 0.f;
-        for (int w = 0; w < kWarps; ++w) sum += red[w * G * (D + 1) + i];
-        const int g = i / (D + 1), d = i % (D + 1);
-        if (d < D) outp[g * (D + 2) + d] = sum;
-        else outp[g * (D + 2) + D + 1] = sum;
+}
+
+template <int D, int G>
+__device__ __forceinline__ void accum_parent_mma(const unsigned char* blk, int C, int jb, int j0,
+                                                 int nrow, const unsigned char* flag,
+                                                 const float* s, int CH, float (&acc)[D / 16][4]) {
+    const int lane = threadIdx.x & 31;
+    const int tg = lane & 3;
+    const uint32_t base = smem_u32(blk);
+    // ldmatrix.x4: lanes 8j..8j+7 address the rows of 8x8 tile j = (rows + 8 (j >> 1),
+    // dims + 8 (j & 1)) of the 16 x 16 step, so registers 0..3 are the A fragment
+    const int lrow = (lane & 7) + ((lane >> 4) << 3);
+    const int ldim = ((lane >> 3) & 1) * 8;
+    for (int k0 = 0; k0 < C; k0 += 16) {
+        uint32_t bh[2], bl[2];
+        weight_frags<G>(s, flag, CH, jb - j0, k0, nrow, bh, bl);
+        // rows past nrow hold other nodes' rows or stale data: their V elements are
+        // masked to zero so that a weight of zero never meets a non-finite value
+        uint32_t m01 = 0xffffffffu, m89 = 0xffffffffu;
+        if (k0 + 16 > nrow) {
+            const int c = k0 + 2 * tg;
+            m01 = (c < nrow ? 0x0000ffffu : 0u) | (c + 1 < nrow ? 0xffff0000u : 0u);
+            m89 = (c + 8 < nrow ? 0x0000ffffu : 0u) | (c + 9 < nrow ? 0xffff0000u : 0u);
+        }
+        const int row = k0 + lrow;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            const int d0 = mt * 16 + ldim;
+            const uint32_t addr = base + swz_off(d0 >> 6, row, (d0 & 63) >> 3, C);
+            uint32_t a0, a1, a2, a3;
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                         : "r"(addr)
+                         : "memory");
+            a0 &= m01;
+            a1 &= m01;
+            a2 &= m89;
+            a3 &= m89;
+            mma_bf16_16816(acc[mt], a0, a1, a2, a3, bh[0], bh[1]);
+            mma_bf16_16816(acc[mt], a0, a1, a2, a3, bl[0], bl[1]);
+        }
     }
-    if (threadIdx.x < G) outp[threadIdx.x * (D + 2) + D] = fm[threadIdx.x];
+}
+
+// Writes each warp's tensor-core accumulators to red[warp][g][d] and finishes the
+// partial record.
+template <int D, int G>
+__device__ __forceinline__ void finish_partial_mma(float (&acc)[D / 16][4], float* lsum,
+                                                   const float* fm, float* red, float* outp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gi = lane >> 2, tg = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int g = 2 * tg + j;
+        if (g < G) {
+            float* row = red + (warp * G + g) * (D + 1);
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                row[mt * 16 + gi] = acc[mt][j];
+                row[mt * 16 + gi + 8] = acc[mt][2 + j];
+            }
+        }
+    }
+    partial_tail<D, G>(lsum, fm, red, outp);
 }
 
 __device__ __forceinline__ void write_empty_partial(float* outp, int G, int D) {
@@ -853,11 +1018,16 @@ __device__ __forceinline__ void cluster_wait() {
 // the last of them merges every partial of the unit into the output.
 // Each warp takes every kWarps-th parent group of the chunk; its K blocks and
 // then its V blocks stream through its ring, so V loads overlap the selection.
+// SW kernels (bf16, d = 128, C a multiple of 16) stage the groups through the
+// swizzled tensor maps of `maps` (the maps of this launch's level) and accumulate
+// values on the tensor cores; the others use plain bulk copies and fp32 FMAs.
 // ----------------------------------------------------------------------------
-template <typename T, int D, int G, bool L0>
-__global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkView wv, QueryView qv,
-                                                            int level, int CH, int NA, int nsw) {
-    extern __shared__ __align__(128) unsigned char smem[];
+template <typename T, int D, int G, bool L0, bool SW>
+__global__ void __launch_bounds__(kThreads, 2)
+    level_kernel(TreeView tv, WorkView wv, QueryView qv, const __grid_constant__ KVMaps maps,
+                 int level, int CH, int NA, int nsw) {
+    static_assert(!SW || kSwzCapable<T, D>, "swizzled staging is bf16, d = 128 only");
+    extern __shared__ __align__(1024) unsigned char smem[];
     if constexpr (L0) {
         // CTAs past the attention grid re-pool the ancestors of each sequence's newest
         // token (one CTA per sequence and KV head); nothing here reads them
@@ -897,6 +1067,14 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
     unsigned char* ring = smem + SL.ring;
     float* red = reinterpret_cast<float*>(smem + SL.red);   // reuses the ring after the last block
     float* fm = reinterpret_cast<float*>(misc + kMiscFloat);
+    if constexpr (SW) {
+        // the swizzle pattern assumes 1024-byte aligned slots; every CTA of the launch
+        // sees the same base, so all of them return here together
+        if (smem_u32(ring) & 1023u) {
+            if (threadIdx.x == 0) set_status(wv.status, kStatusLayout);
+            return;
+        }
+    }
 
     const int unit = blockIdx.y;
     const int split = blockIdx.x;
@@ -1009,7 +1187,10 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
     auto issue = [&](int q) {
         const int i = q < nk ? q : q - nk;
         const int jb = j0 + (warp + kWarps * i) * C;
-        ring_issue<T, D>(R, q, q < nk ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
+        if constexpr (SW)
+            ring_issue_map(R, q, q < nk ? &maps.k : &maps.v, group_first(jb), kvh, b, C);
+        else
+            ring_issue<T, D>(R, q, q < nk ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
     };
     if (identity && rs == D && threadIdx.x == 0 && j1 > j0) {
         // the first scored level was not prefetched by a level above: its chunk
@@ -1048,8 +1229,9 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
             const int nch = min(C, j0 + n_sc - jb);
             const int next_jb = (i + 1 < nw) ? jb + kWarps * C : -1;
             if (nch > 0)
-                score_parent<T, D, G, !L0>(blk, jb, next_jb, j0, nch, group_first(jb), wv.rope, p_q,
-                                           rc4, qsm, tv.scale, s, key, nodes, CH);
+                score_parent<T, D, G, !L0, SW>(blk, C, jb, next_jb, j0, nch, group_first(jb),
+                                               wv.rope, p_q, rc4, qsm, tv.scale, s, key, nodes,
+                                               CH);
             __syncwarp();
             if (lane == 0 && i + nsw < nk + nw) issue(i + nsw);
         }
@@ -1116,23 +1298,41 @@ __global__ void __launch_bounds__(kThreads, 2) level_kernel(TreeView tv, WorkVie
     float lsum[G];
     // (scratch: the histogram area; the ring, and so red, still holds V blocks)
     softmax_weights<G>(s, n_sc, L0 ? nullptr : flag, CH, reinterpret_cast<float*>(hist), fm, lsum);
-    float2 acc[G][V2];
+    if constexpr (SW) {
+        float acc[D / 16][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        for (int i = 0; i < nw; ++i) {
+            const int q = nk + i;
+            const unsigned char* blk = ring_wait(R, q);
+            const int jb = j0 + (warp + kWarps * i) * C;
+            const int nrow = min(C, j0 + n_sc - jb);
+            if (nrow > 0 && fm[0] > -INFINITY)
+                accum_parent_mma<D, G>(blk, C, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
+            __syncwarp();
+            if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
+        }
+        __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
+        finish_partial_mma<D, G>(acc, lsum, fm, red, outp);
+    } else {
+        float2 acc[G][V2];
 #pragma unroll
-        for (int e = 0; e < V2; ++e) acc[g][e] = make_float2(0.f, 0.f);
-    for (int i = 0; i < nw; ++i) {
-        const int q = nk + i;
-        const unsigned char* blk = ring_wait(R, q);
-        const int jb = j0 + (warp + kWarps * i) * C;
-        const int nrow = min(C, j0 + n_sc - jb);
-        if (nrow > 0 && fm[0] > -INFINITY)
-            accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
-        __syncwarp();
-        if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < V2; ++e) acc[g][e] = make_float2(0.f, 0.f);
+        for (int i = 0; i < nw; ++i) {
+            const int q = nk + i;
+            const unsigned char* blk = ring_wait(R, q);
+            const int jb = j0 + (warp + kWarps * i) * C;
+            const int nrow = min(C, j0 + n_sc - jb);
+            if (nrow > 0 && fm[0] > -INFINITY)
+                accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
+            __syncwarp();
+            if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
+        }
+        __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
+        finish_partial<T, D, G>(acc, lsum, fm, red, outp);
     }
-    __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
-    finish_partial<T, D, G>(acc, lsum, fm, red, outp);
 
     if (L0) {
         if (split == 0 && threadIdx.x == 0) {
@@ -1172,28 +1372,38 @@ static size_t level_smem(int C, int k, int splits, bool l0) {
     return smem_layout(G, D, CH, k, C, l0 ? 0 : C * k, kWarps * nsw * C * D * (int)sizeof(T)).total;
 }
 
-template <typename T, int D, int G>
-static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
-    const size_t sm = level_smem<T, D, G>(C, k, SPL, false);
-    const size_t sm0 = level_smem<T, D, G>(C, k, NS0, true);
-    if (sm > 227 * 1024 || sm0 > 227 * 1024) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(level_kernel<T, D, G, false>,
+template <typename T, int D, int G, bool SW>
+static cudaError_t prepare_variant(size_t sm, size_t sm0, int SPL) {
+    cudaError_t e = cudaFuncSetAttribute(level_kernel<T, D, G, false, SW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     if (SPL > 8) {
-        e = cudaFuncSetAttribute(level_kernel<T, D, G, false>,
+        e = cudaFuncSetAttribute(level_kernel<T, D, G, false, SW>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
     }
     const size_t walk = ancestor_walk_smem(kMaxLevels, D);
-    return cudaFuncSetAttribute(level_kernel<T, D, G, true>,
+    return cudaFuncSetAttribute(level_kernel<T, D, G, true, SW>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(sm0 > walk ? sm0 : walk));
 }
 
 template <typename T, int D, int G>
-static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, const QueryView& qv,
-                                      cudaStream_t s, const ProfHook* prof) {
+static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
+    const size_t sm = level_smem<T, D, G>(C, k, SPL, false);
+    const size_t sm0 = level_smem<T, D, G>(C, k, NS0, true);
+    if (sm > 227 * 1024 || sm0 > 227 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = prepare_variant<T, D, G, false>(sm, sm0, SPL);
+    if constexpr (kSwzCapable<T, D>)
+        if (e == cudaSuccess) e = prepare_variant<T, D, G, true>(sm, sm0, SPL);
+    return e;
+}
+
+template <typename T, int D, int G, bool SW>
+static cudaError_t select_attend_variant(const TreeView& tv, const WorkView& wv,
+                                         const QueryView& qv, cudaStream_t s, const ProfHook* prof,
+                                         const KVMaps* maps) {
+    static const KVMaps kNoMaps = {};
     const int CH = chunk_cap(tv.k, wv.SPL, tv.C), CH0 = chunk_cap(tv.k, wv.NS0, tv.C);
     const int NA = tv.C * tv.k;
     const int nsw = slots_per_warp(tv.C, D, (int)sizeof(T));
@@ -1215,8 +1425,8 @@ static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, co
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         prof_mark(prof, level, true, s);
-        cudaError_t e =
-            cudaLaunchKernelEx(&cfg, level_kernel<T, D, G, false>, tv, wv, qv, level, CH, NA, nsw);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, level_kernel<T, D, G, false, SW>, tv, wv, qv,
+                                           SW ? maps[level] : kNoMaps, level, CH, NA, nsw);
         prof_mark(prof, level, false, s);
         if (e != cudaSuccess) return e;
     }
@@ -1233,10 +1443,26 @@ static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, co
     cfg0.attrs = attr0;
     cfg0.numAttrs = 1;
     prof_mark(prof, 0, true, s);
-    cudaError_t e0 = cudaLaunchKernelEx(&cfg0, level_kernel<T, D, G, true>, tv, wv, qv, 0, CH0, 0, nsw);
+    cudaError_t e0 = cudaLaunchKernelEx(&cfg0, level_kernel<T, D, G, true, SW>, tv, wv, qv,
+                                        SW ? maps[0] : kNoMaps, 0, CH0, 0, nsw);
     prof_mark(prof, 0, false, s);
     if (e0 != cudaSuccess) return e0;
     return cudaGetLastError();
+}
+
+// maps: the tensor maps of every level when the tree stages through them (bf16,
+// d = 128, C a multiple of 16), else null.
+template <typename T, int D, int G>
+static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, const QueryView& qv,
+                                      cudaStream_t s, const ProfHook* prof, const KVMaps* maps) {
+    if constexpr (kSwzCapable<T, D>) {
+        if (maps) {
+            if (tv.C % 16 != 0 || tv.n_levels > kMaxLevels) return cudaErrorInvalidValue;
+            return select_attend_variant<T, D, G, true>(tv, wv, qv, s, prof, maps);
+        }
+    }
+    if (maps) return cudaErrorInvalidValue;
+    return select_attend_variant<T, D, G, false>(tv, wv, qv, s, prof, nullptr);
 }
 
 #define RECSA_DISPATCH_TDG(dtype, D, G, FN, ...)                                          \
@@ -1273,8 +1499,9 @@ cudaError_t prepare_kernels(int dtype, int D, int G, int SPL, int NS0, int C, in
 }
 
 cudaError_t launch_select_attend(const TreeView& tv, const WorkView& wv, const QueryView& qv,
-                                 int dtype, cudaStream_t s, const ProfHook* prof) {
-    RECSA_DISPATCH_TDG(dtype, tv.D, tv.G, select_attend_impl, tv, wv, qv, s, prof);
+                                 int dtype, cudaStream_t s, const ProfHook* prof,
+                                 const KVMaps* maps) {
+    RECSA_DISPATCH_TDG(dtype, tv.D, tv.G, select_attend_impl, tv, wv, qv, s, prof, maps);
 }
 
 }  // namespace recsa
