@@ -99,15 +99,24 @@ __device__ __forceinline__ uint32_t swz_off(int half, int row, int chunk, int C)
 // shared-memory layout of the select/attend kernels
 // ----------------------------------------------------------------------------
 struct Smem {
-    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, misc, bars, ring, red, total;
+    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, gs, misc, bars, ring, red, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
-// CH: entries per CTA chunk; NA: largest list (C*k), 0 when no key exchange is
-// needed; ring_bytes: the warps' staging slots.  The reduction buffer reuses the
-// ring once every block has been consumed.
-__host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, int NA,
+// Words of the cluster selection's global histogram held by each of `csize` CTAs
+// (a multiple of 4, so a 16-byte group of words has one owner).
+__host__ __device__ inline int gs_words(int csize) {
+    return ((1024 + csize - 1) / csize + 3) & ~3;
+}
+constexpr int kSelCand = 384;   // candidates of the cluster selection's boundary bin
+
+// CH: entries per CTA chunk; NA: largest list (C*k), 0 at level 0 (no selection);
+// gsw: the CTA's slice of the cluster histogram (0 at level 0); ring_bytes: the
+// warps' staging slots.  The reduction buffer reuses the ring once every block has
+// been consumed.  mkey holds the exchanged keys of the heavy-tie path, or the
+// published and gathered candidates of the cluster selection.
+__host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, int NA, int gsw,
                                             int ring_bytes) {
     Smem L;
     size_t o = 0;
@@ -118,9 +127,11 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
     L.nodes = o; o = align16(o + sizeof(int) * CH);
     L.flag = o;  o = align16(o + sizeof(unsigned char) * CH);
     L.par = o;   o = align16(o + sizeof(int) * k);
-    L.mkey = o;  o = align16(o + sizeof(uint32_t) * NA);
+    const int mk = NA > 0 && NA < 4 * kSelCand ? 4 * kSelCand : NA;
+    L.mkey = o;  o = align16(o + sizeof(uint32_t) * mk);
     L.hist = o;  o = align16(o + sizeof(uint32_t) * 1024);   // >= kSelBins / 2, radix 512
-    L.misc = o;  o = align16(o + sizeof(int) * 64);
+    L.gs = o;    o = align16(o + sizeof(uint32_t) * gsw);
+    L.misc = o;  o = align16(o + sizeof(int) * 128);
     L.bars = o;  o = align16(o + sizeof(uint64_t) * kWarps * 2);
     o = (o + 1023) & ~size_t(1023);   // swizzled slots need 1024-byte alignment
     L.ring = o;
@@ -133,7 +144,19 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
 
 // misc slots
 enum { kMiscDigit = 0, kMiscAbove = 1, kMiscCount = 2, kMiscScan = 4 /* kWarps+1 */,
-       kMiscFloat = 16 /* 2*G floats */, kMiscLast = 40, kMiscN = 41 };
+       kMiscFloat = 16 /* 2*G floats */, kMiscLast = 40, kMiscN = 41,
+       // cluster selection: published counts, gathered counts (one per CTA), scalars
+       kMiscPubC = 48, kMiscPubA = 49, kMiscSB = 50, kMiscSBAbove = 51, kMiscMemN = 52,
+       kMiscTk = 53, kMiscTj = 54, kMiscGC = 64 /* 16 */, kMiscGA = 80 /* 16 */ };
+
+// Split cluster barrier: arrive (release) and, later, wait (acquire); every thread
+// of every CTA of the cluster takes both, in this order.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // ----------------------------------------------------------------------------
 // block-wide primitives (kThreads threads)
@@ -334,8 +357,33 @@ __device__ void block_select_ranks_short(const uint32_t* keys, int n, uint32_t T
 // hist: kSelBins / 2 words.
 constexpr int kSelBits = 11;
 constexpr int kSelBins = 1 << kSelBits;
-constexpr int kSelCand = 384;
 enum { kMiscCand = 3, kMiscT = 13, kMiscNeedEq = 14, kMiscCntEq = 15 };
+
+// Given each thread's BPT bin counts in descending bin order (thread t owns bins
+// kSelBins-1-BPT*t-u), finds the bin holding the K-th largest key: misc[kMiscDigit]
+// = the bin, misc[kMiscAbove] = keys in higher bins, misc[kMiscCount] = its keys.
+template <int BPT>
+__device__ __forceinline__ void find_boundary_bin(const uint32_t (&cnt8)[BPT], int K, int* misc) {
+    int tot = 0;
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) tot += (int)cnt8[u];
+    int all;
+    const int excl = block_excl_scan(tot, misc + kMiscScan, all);
+    if (excl < K && K <= excl + tot) {
+        int run = excl;
+#pragma unroll
+        for (int u = 0; u < BPT; ++u) {
+            if (run + (int)cnt8[u] >= K) {
+                misc[kMiscDigit] = kSelBins - 1 - BPT * (int)threadIdx.x - u;
+                misc[kMiscAbove] = run;
+                misc[kMiscCount] = (int)cnt8[u];
+                break;
+            }
+            run += (int)cnt8[u];
+        }
+    }
+    __syncthreads();
+}
 
 template <typename Fn>
 __device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* misc, int lo, int hi,
@@ -356,29 +404,12 @@ __device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* m
     __syncthreads();
     // thread t owns bins kSelBins-1-BPT*t-u, u = 0..BPT-1 (descending key order)
     uint32_t cnt8[BPT];
-    int tot = 0;
 #pragma unroll
     for (int u = 0; u < BPT; ++u) {
         const int bin = kSelBins - 1 - BPT * tid - u;
         cnt8[u] = (hist[bin >> 1] >> (16 * (bin & 1))) & 0xFFFFu;
-        tot += (int)cnt8[u];
     }
-    int all;
-    const int excl = block_excl_scan(tot, misc + kMiscScan, all);
-    if (excl < K && K <= excl + tot) {
-        int run = excl;
-#pragma unroll
-        for (int u = 0; u < BPT; ++u) {
-            if (run + (int)cnt8[u] >= K) {
-                misc[kMiscDigit] = kSelBins - 1 - BPT * tid - u;
-                misc[kMiscAbove] = run;
-                misc[kMiscCount] = (int)cnt8[u];
-                break;
-            }
-            run += (int)cnt8[u];
-        }
-    }
-    __syncthreads();
+    find_boundary_bin<BPT>(cnt8, K, misc);
     const uint32_t bd = (uint32_t)misc[kMiscDigit];
     const int need = K - misc[kMiscAbove];   // keys to take from bin bd: 1..cnt
     const int cnt = misc[kMiscCount];
@@ -447,6 +478,183 @@ __device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* m
         block_select_ranks_short(mkey, M, T, need_eq, cnt_eq, lo, hi, misc, mark);
     else
         block_select_ranks(mkey, M, T, need_eq, cnt_eq, lo, hi, misc, mark);
+}
+
+// ----------------------------------------------------------------------------
+// Exact top-K (0 < K < M) over a cluster.  The M keys of a list are spread over the
+// csize CTAs of the cluster: CTA r holds, in its `key` array, the n_loc keys of
+// the contiguous slice that starts at list position j0 = r * chunk.  Every CTA
+// finds the same threshold (T, jT), the K-th entry in the order (key descending,
+// list position ascending); entry j is selected when key > T, or key == T and
+// j <= jT.  mark(j, rank) is called for this CTA's selected entries, rank = the
+// entry's position among all selected entries in list order.
+//  1. Each CTA histograms the leading kSelBits bits of its keys (lh, zeroed by the
+//     caller) and adds its non-zero words into the global histogram, whose words
+//     are spread over the CTAs (gsw words each, zeroed by the caller before a
+//     cluster arrive that the caller's wait completed): distributed shared memory
+//     atomics.  A cluster barrier follows.
+//  2. Every CTA reads the global histogram and finds the bin bd holding the K-th
+//     key.  A bin of more than kSelCand keys (heavy ties) returns false here, in
+//     every CTA alike, and the caller runs the exchange-and-select path instead.
+//  3. Each CTA publishes the (key, position) pairs of its keys in bd and its count
+//     of keys above bd; after a second barrier every CTA gathers all candidates
+//     (then arrives on the cluster barrier that the caller waits on before exit).
+//     The threshold follows from a 256-bin histogram of the candidates' next 8 key
+//     bits and an exact rank of the few candidates in the boundary sub-bin.
+//  4. A selected entry's rank is the count of selected entries in the CTAs before
+//     this one (their counts above bd plus their selected candidates) plus its
+//     rank within this CTA.
+// ----------------------------------------------------------------------------
+template <typename Fn>
+__device__ bool cluster_select(const uint32_t* key, int n_loc, int j0, int K, int csize, int crank,
+                               int gsw, uint32_t* lh, uint32_t* gs, uint2* pub, uint2* all,
+                               int* misc, Fn mark) {
+    constexpr int SH = 32 - kSelBits;
+    constexpr int BPT = kSelBins / kThreads;
+    constexpr int W = kSelBins / 2;   // histogram words, two 16-bit counts each
+    static_assert(W == 4 * kThreads && kThreads == 256, "one 16-byte word group per thread");
+    cg::cluster_group cluster = cg::this_cluster();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // 1. local histogram, then its non-zero words into their owners' slices
+    for (int i = tid; i < n_loc; i += kThreads) {
+        const uint32_t dig = key[i] >> SH;
+        atomicAdd(&lh[dig >> 1], 1u << (16 * (dig & 1)));
+    }
+    __syncthreads();
+    {
+        const uint4 w = *reinterpret_cast<const uint4*>(lh + 4 * tid);
+        if (w.x | w.y | w.z | w.w) {
+            uint32_t* dst = cluster.map_shared_rank(gs, (4 * tid) / gsw) + (4 * tid) % gsw;
+            if (w.x) atomicAdd(dst, w.x);
+            if (w.y) atomicAdd(dst + 1, w.y);
+            if (w.z) atomicAdd(dst + 2, w.z);
+            if (w.w) atomicAdd(dst + 3, w.w);
+        }
+    }
+    cluster.sync();
+
+    // 2. the global histogram: thread t owns bins kSelBins-1-BPT*t-u, the words
+    //    from W-4-4t (bin b: word b/2, high half when b is odd)
+    {
+        const int w0 = W - 4 - 4 * tid;
+        const uint4 w = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(gs, w0 / gsw) + w0 % gsw);
+        const uint32_t ws[4] = {w.w, w.z, w.y, w.x};
+        uint32_t cnt8[BPT];
+#pragma unroll
+        for (int u = 0; u < BPT; ++u) cnt8[u] = (ws[u >> 1] >> (16 * (1 - (u & 1)))) & 0xFFFFu;
+        find_boundary_bin<BPT>(cnt8, K, misc);
+    }
+    const uint32_t bd = (uint32_t)misc[kMiscDigit];
+    const int cnt = misc[kMiscCount];
+    if (cnt > kSelCand) return false;
+    const int need = K - misc[kMiscAbove];   // 1..cnt
+
+    // 3. this CTA's candidates and its count above bd, for the other CTAs
+    int my_above = 0;
+    for (int i0 = 0; i0 < n_loc; i0 += kThreads) {
+        const int i = i0 + tid;
+        const uint32_t kk = i < n_loc ? key[i] : 0u;
+        const uint32_t dig = kk >> SH;
+        const bool in = i < n_loc && dig == bd;
+        my_above += (i < n_loc && dig > bd) ? 1 : 0;
+        const unsigned bal = __ballot_sync(kFull, in);
+        if (bal) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&misc[kMiscPubC], __popc(bal));
+            base = __shfl_sync(kFull, base, 0);
+            if (in) pub[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(kk, (uint32_t)(j0 + i));
+        }
+    }
+    my_above = (int)__reduce_add_sync(kFull, (unsigned)my_above);
+    if (lane == 0 && my_above) atomicAdd(&misc[kMiscPubA], my_above);
+    cluster.sync();
+    if (tid < csize) {
+        const int* rm = cluster.map_shared_rank(misc, tid);
+        misc[kMiscGC + tid] = rm[kMiscPubC];
+        misc[kMiscGA + tid] = rm[kMiscPubA];
+    }
+    uint32_t* sub = lh;   // free since step 1: sub-bin counts, then the member list
+    sub[tid] = 0u;
+    if (tid == 0) misc[kMiscMemN] = 0;
+    __syncthreads();
+    for (int idx = tid; idx < cnt; idx += kThreads) {
+        int r = 0, off = 0;
+        while (r < csize - 1 && idx >= off + misc[kMiscGC + r]) off += misc[kMiscGC + r++];
+        const uint2 c = cluster.map_shared_rank(pub, r)[idx - off];
+        all[idx] = c;
+        atomicAdd(&sub[(c.x >> (SH - 8)) & 255u], 1u);
+    }
+    int base_above = 0;
+    for (int r = 0; r < crank; ++r) base_above += misc[kMiscGA + r];
+    __syncthreads();
+    cluster_arrive();   // remote reads done; the caller waits before exit
+
+    // threshold: the sub-bin (next 8 bits) holding the need-th candidate ...
+    {
+        const int c = (int)sub[255 - tid];
+        int tot;
+        const int ex = block_excl_scan(c, misc + kMiscScan, tot);
+        if (ex < need && need <= ex + c) {
+            misc[kMiscSB] = 255 - tid;
+            misc[kMiscSBAbove] = ex;
+        }
+        __syncthreads();
+    }
+    const uint32_t sb = (uint32_t)misc[kMiscSB];
+    const int need2 = need - misc[kMiscSBAbove];
+    // ... and the exact rank of each candidate in that sub-bin among the others there
+    for (int i0 = 0; i0 < cnt; i0 += kThreads) {
+        const int idx = i0 + tid;
+        const bool in = idx < cnt && ((all[idx].x >> (SH - 8)) & 255u) == sb;
+        const unsigned bal = __ballot_sync(kFull, in);
+        if (bal) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&misc[kMiscMemN], __popc(bal));
+            base = __shfl_sync(kFull, base, 0);
+            if (in) sub[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)idx;
+        }
+    }
+    __syncthreads();
+    const int nm = misc[kMiscMemN];
+    for (int mi = warp; mi < nm; mi += kWarps) {
+        const uint2 me = all[sub[mi]];
+        int gt = 0;
+        for (int o = lane; o < nm; o += 32) {
+            const uint2 x = all[sub[o]];
+            gt += (x.x > me.x || (x.x == me.x && x.y < me.y)) ? 1 : 0;
+        }
+        gt = (int)__reduce_add_sync(kFull, (unsigned)gt);
+        if (lane == 0 && gt == need2 - 1) {
+            misc[kMiscTk] = (int)me.x;
+            misc[kMiscTj] = (int)me.y;
+        }
+    }
+    __syncthreads();
+    const uint32_t T = (uint32_t)misc[kMiscTk], jT = (uint32_t)misc[kMiscTj];
+
+    // 4. ranks: selected candidates of the CTAs before this one, then this CTA's
+    int sc = 0;
+    for (int idx = tid; idx < cnt; idx += kThreads) {
+        const uint2 c = all[idx];
+        sc += (c.y < (uint32_t)j0 && (c.x > T || (c.x == T && c.y <= jT))) ? 1 : 0;
+    }
+    int sel_before;
+    block_excl_scan(sc, misc + kMiscScan, sel_before);
+    const int ipt = (n_loc + kThreads - 1) / kThreads;
+    const int i0 = tid * ipt, i1 = min(n_loc, i0 + ipt);
+    int cs = 0;
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t kk = key[i];
+        cs += (kk > T || (kk == T && (uint32_t)(j0 + i) <= jT)) ? 1 : 0;
+    }
+    int tot;
+    int r = base_above + sel_before + block_excl_scan(cs, misc + kMiscScan, tot);
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t kk = key[i];
+        if (kk > T || (kk == T && (uint32_t)(j0 + i) <= jT)) mark(j0 + i, r++);
+    }
+    return true;
 }
 
 // ----------------------------------------------------------------------------
@@ -627,12 +835,9 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int C, in
                 PairLoad<T, PPL>::get(row + kHalf + off, kh);
             }
             const float4* rc = rc4 + cr * (H / 2) + cl;
-            float2 alo[G], ahi[G];
+            float2 acc[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                alo[g] = make_float2(0.f, 0.f);
-                ahi[g] = make_float2(0.f, 0.f);
-            }
+            for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int w = 0; w < CPL; ++w) {
                 const float4 cs = rc[w * LPK];   // (cos v, cos v+1, sin v, sin v+1) of c * theta
@@ -643,13 +848,12 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int C, in
                 const float2 kb = __ffma2_rn(kl[w], si, __fmul2_rn(kh[w], co));
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    alo[g] = __ffma2_rn(qlo[g][w], ka, alo[g]);
-                    ahi[g] = __ffma2_rn(qhi[g][w], kb, ahi[g]);
+                    acc[g] = __ffma2_rn(qlo[g][w], ka, acc[g]);
+                    acc[g] = __ffma2_rn(qhi[g][w], kb, acc[g]);
                 }
             }
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-                v[u * G + g] = (alo[g].x + ahi[g].x) + (alo[g].y + ahi[g].y);
+            for (int g = 0; g < G; ++g) v[u * G + g] = acc[g].x + acc[g].y;
         }
         if constexpr (RS) {
             reduce_scatter<NV, LPK>(v, cl);
@@ -1005,12 +1209,6 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
     }
 }
 
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 
 // ----------------------------------------------------------------------------
 // level l >= 1: score + RoPE + TopK + summaries (cluster of SPL CTAs per unit)
@@ -1051,7 +1249,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int k = tv.k, C = tv.C, lgC = tv.lgC, K1 = k - 1, NL = wv.NL;
     const int nsplit = L0 ? wv.NS0 : wv.SPL;
     const int slot_bytes = C * kRow;
-    const Smem SL = smem_layout(G, D, CH, k, C, L0 ? 0 : NA, kWarps * nsw * slot_bytes);
+    const int gsw = L0 ? 0 : gs_words(nsplit);
+    const Smem SL = smem_layout(G, D, CH, k, C, L0 ? 0 : NA, gsw, kWarps * nsw * slot_bytes);
     float* qsm = reinterpret_cast<float*>(smem + SL.qsm);
     float4* rc4 = reinterpret_cast<float4*>(smem + SL.rc4);
 
@@ -1062,6 +1261,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int* par = reinterpret_cast<int*>(smem + SL.par);
     uint32_t* mkey = reinterpret_cast<uint32_t*>(smem + SL.mkey);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + SL.hist);
+    uint32_t* gs = reinterpret_cast<uint32_t*>(smem + SL.gs);
     int* misc = reinterpret_cast<int*>(smem + SL.misc);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bars);
     unsigned char* ring = smem + SL.ring;
@@ -1200,6 +1400,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (lane == 0)
         for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
+    if (!L0) {
+        // the selection's histograms and published counts start at zero in every CTA
+        // of the cluster before any CTA adds into them (waited on after the scores)
+        for (int i = threadIdx.x; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
+        for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
+        if (threadIdx.x == 0) misc[kMiscPubC] = misc[kMiscPubA] = 0;
+        __syncthreads();
+        cluster_arrive();
+    }
 
     // 1. scores of the chunk
     if (pre) {
@@ -1242,23 +1451,41 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (L0) __syncthreads();
 
     if (!L0) {
-        // 2. every CTA's keys in list order (list position = merged index)
         cg::cluster_group cluster = cg::this_cluster();
         const int csize = (int)cluster.num_blocks();
         const int crank = (int)cluster.block_rank();
-        cluster.sync();
         const int M = nA - 1;
-        for (int r = 0; r < csize; ++r) {
-            const int lo = r * chunk, hi = min(M, lo + chunk);
-            if (hi <= lo) break;
-            const uint32_t* rk = cluster.map_shared_rank(key, r);
-#pragma unroll 4
-            for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
-        }
-        cluster_arrive();   // remote reads done; matched by cluster_wait() before exit
+        cluster_wait();   // every CTA's zeroed histograms (and, later, keys) are in place
         __syncthreads();
-
-        // 3. exact top-(k-1) over all M keys; this CTA writes S for its entries
+        // 2. exact top-(k-1) over all M keys; this CTA writes S for its entries
+        auto mark = [&](int i, int r) {
+            const int node = nodes[i - j0];
+            sel_ws[r] = node;
+            if (sel_usr) sel_usr[r] = node;
+            flag[i - j0] = 1;
+        };
+        bool done = true;
+        if (K1 > 0) {   // k = 1: only the current node is selected
+            uint2* pub = reinterpret_cast<uint2*>(mkey);
+            done = cluster_select(key, n_sc, j0, K1, csize, crank, gsw, hist, gs, pub,
+                                  pub + kSelCand, misc, mark);
+        } else {
+            cluster_arrive();
+        }
+        if (!done) {
+            // heavy ties: every CTA's keys in list order (list position = merged
+            // index), then the block-wide select (same set)
+            for (int r = 0; r < csize; ++r) {
+                const int lo = r * chunk, hi = min(M, lo + chunk);
+                if (hi <= lo) break;
+                const uint32_t* rk = cluster.map_shared_rank(key, r);
+#pragma unroll 4
+                for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
+            }
+            cluster_arrive();   // remote reads done; matched by cluster_wait() before exit
+            __syncthreads();
+            select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, mark);
+        }
         const T* nk;
         const T* nv;
         int64_t nrs;
@@ -1271,13 +1498,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             nv = level_v<T>(tv, level - 1, b, kvh);
             nrs = D;
         }
-        if (K1 > 0)   // k = 1: only the current node is selected
-            select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, [&](int i, int r) {
-                const int node = nodes[i - j0];
-                sel_ws[r] = node;
-                if (sel_usr) sel_usr[r] = node;
-                flag[i - j0] = 1;
-            });
         if (crank == 0 && threadIdx.x == 0) {
             const int64_t cur = apow(t, level, C, lgC);
             sel_ws[K1] = (int)cur;
@@ -1369,7 +1589,9 @@ template <typename T, int D, int G>
 static size_t level_smem(int C, int k, int splits, bool l0) {
     const int CH = chunk_cap(k, splits, C);
     const int nsw = slots_per_warp(C, D, (int)sizeof(T));
-    return smem_layout(G, D, CH, k, C, l0 ? 0 : C * k, kWarps * nsw * C * D * (int)sizeof(T)).total;
+    return smem_layout(G, D, CH, k, C, l0 ? 0 : C * k, l0 ? 0 : gs_words(splits),
+                       kWarps * nsw * C * D * (int)sizeof(T))
+        .total;
 }
 
 template <typename T, int D, int G, bool SW>
