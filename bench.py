@@ -28,31 +28,31 @@ sys.path.insert(0, ROOT)
 
 METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
 
-# DRAM bytes (read + write) per launch of the level-1 select/attend kernel from one
-# ncu capture at batch 1 (profiles/level_kernels_decode524k_b1.md); a launch covers
+# DRAM bytes (read + write) per launch of the select/attend pass kernel from one ncu
+# capture at batch 1 (profiles/pass_kernel_decode524k_b1.md); a launch covers
 # batch x 8 independent units, so the batch-B figure is B times this.  Valid only
 # for the kernel sources it was taken from: any edit to them turns it into null.
-TRAFFIC_LEVEL1_B1 = {"bytes": 33_696_768 + 768,
-                     "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
-                                 "long_context_recsa_b200/csrc/recsa_internal.cuh",
-                                 "long_context_recsa_b200/csrc/pool.cuh"],
-                     "sha256": "6097bdea1e6b5080d3675c9c800bcf7587188a87301373798545b15f22399bc7"}
+TRAFFIC_PASS_B1 = {"bytes": None,
+                   "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
+                               "long_context_recsa_b200/csrc/recsa_internal.cuh",
+                               "long_context_recsa_b200/csrc/pool.cuh"],
+                   "sha256": ""}
 
 
 def captured_traffic(kernel: str, batch: int):
     """Per-launch DRAM traffic of `kernel` at this batch, or None when no capture of
     the current sources exists."""
     import hashlib
-    if kernel != "level1_kernel":
+    if kernel != "pass_kernel" or TRAFFIC_PASS_B1["bytes"] is None:
         return None
     h = hashlib.sha256()
     here = os.path.dirname(os.path.abspath(__file__))
-    for f in TRAFFIC_LEVEL1_B1["sources"]:
+    for f in TRAFFIC_PASS_B1["sources"]:
         with open(os.path.join(here, f), "rb") as fh:
             h.update(fh.read())
-    if h.hexdigest() != TRAFFIC_LEVEL1_B1["sha256"]:
+    if h.hexdigest() != TRAFFIC_PASS_B1["sha256"]:
         return None
-    return TRAFFIC_LEVEL1_B1["bytes"] * batch
+    return TRAFFIC_PASS_B1["bytes"] * batch
 HBM_NOMINAL_GBS = 8000.0
 
 # workload: 524K decode, B = 4 (and the 4096-query prefill chunk at 524K)
@@ -270,7 +270,7 @@ def run_ours(args):
     out = torch.empty_like(qst)
     cnt = torch.zeros(B, Hkv, tree.n_sel_levels + 1, dtype=torch.int32, device=dev)
     prof_ev = {}
-    for which in [0] + list(range(1, tree.n_sel_levels + 1)) + [-1]:
+    for which in [0, -1]:   # the select/attend pass, the append
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(); b_.record()
         prof_ev[which] = (a, b_)
@@ -294,7 +294,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    launches_per_step = 1 + tree.n_sel_levels + 1   # append, levels n..1, level 0
+    launches_per_step = 2   # append, select/attend pass
     step_ms, kern_ms = [], {w: [] for w in prof_ev}
     whiches = list(prof_ev)
 
@@ -333,9 +333,9 @@ def run_ours(args):
     by_step, per_level = step_bytes(counts, k, d * esize, B, Hkv, Hq, d, esize)
     hbm, peak_kind = peaks()
     kern_avg = {w: (sum(v) / len(v) if v else None) for w, v in kern_ms.items()}
-    # dominant kernel: the one with the largest share of the step
-    dom = max((w for w in kern_avg if w >= 0 and kern_avg[w]), key=lambda w: kern_avg[w])
-    dom_bytes = per_level.get(dom, 0)
+    # dominant kernel: the select/attend pass (every level of every unit)
+    dom = 0
+    dom_bytes = sum(per_level.values())
     achieved = dom_bytes / (kern_avg[dom] / 1e3) / 1e9
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": ws,
@@ -346,16 +346,15 @@ def run_ours(args):
         "bytes_per_step": int(by_step),
         "hbm_frac_of_nominal_8TBs": round(by_step / (ms / 1e3) / 1e9 / HBM_NOMINAL_GBS, 4),
         "hbm_frac_of_measured": round(by_step / (ms / 1e3) / 1e9 / hbm, 4),
-        "roofline": {"bound": "hbm", "kernel": f"level{dom}_kernel",
+        "roofline": {"bound": "hbm", "kernel": "pass_kernel",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4),
-                     "traffic": captured_traffic(f"level{dom}_kernel", B),
-                     "traffic_note": "ncu batch-1 capture x batch; includes the L2 prefetch "
-                                     "of the next level's rows (255 x 16 rows x 512 B per unit)",
+                     "traffic": captured_traffic("pass_kernel", B),
+                     "traffic_note": "ncu batch-1 capture x batch",
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": int(dom_bytes),
                      "avg_launch_ms": round(kern_avg[dom], 5)},
-        "kernel_ms": {("append" if w == -1 else f"level{w}"):
+        "kernel_ms": {("append" if w == -1 else "pass"):
                       (round(v, 5) if v else None) for w, v in kern_avg.items()},
         "build_524k": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1)},
         "gpu_launches": launches_per_step * args.steps,

@@ -211,8 +211,8 @@ RECSA_API recsa_status recsa_host_lengths(const recsa_tree* tree, int64_t* lengt
 /* Kernel timing hook.  From the next call on, record CUDA event `start` (a
  * cudaEvent_t, created by the caller with timing enabled) on the call's stream just
  * before the kernel selected by `which` is launched and `stop` just after it:
- *   which = l in [0, n_sel_levels]: the select/attend kernel of level l (0 = the
- *           level-0 attention), in recsa_decode and in each prefill wave;
+ *   which = 0: the select/attend pass kernel (every level of every unit), in
+ *           recsa_decode and in each prefill wave;
  *   which = -1: the append kernel(s) of recsa_append;  -2: the tensor-core product
  *   of recsa_prefill_chunk (the last one of the call).
  * Records use cudaEventRecordExternal, so they also become event nodes when the

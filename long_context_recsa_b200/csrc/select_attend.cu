@@ -1166,11 +1166,12 @@ __device__ __forceinline__ void write_empty_partial(float* outp, int G, int D) {
     }
 }
 
-// Log-sum-exp merge of a unit's partials into its G output heads.  Partials of
-// other CTAs are read through L2 (ld.global.cg).
+// Log-sum-exp merge of a unit's partials into its G output heads, output elements
+// [e0, e1) of the G*D.  Partials of other CTAs are read through L2 (ld.global.cg).
 template <typename T, int D, int G>
 __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL, T* out,
-                             float* wsh /* >= G*(NL*SPL+NS0) */, float* Lsh /* G */) {
+                             float* wsh /* >= G*(NL*SPL+NS0) */, float* Lsh /* G */, int e0,
+                             int e1) {
     const int nls = lstar * SPL;
     const int ns = nls + NS0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1196,7 +1197,7 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
         if (lane == 0) Lsh[g] = L;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    for (int e = e0 + (int)threadIdx.x; e < e1; e += kThreads) {
         const int g = e / D, d = e % D;
         float O = 0.f;
 #pragma unroll 4
@@ -1211,49 +1212,58 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
 
 
 // ----------------------------------------------------------------------------
-// level l >= 1: score + RoPE + TopK + summaries (cluster of SPL CTAs per unit)
-// level 0 (L0 = true): score + softmax partial over A^(0) (NS0 CTAs per unit);
-// the last of them merges every partial of the unit into the output.
-// Each warp takes every kWarps-th parent group of the chunk; its K blocks and
-// then its V blocks stream through its ring, so V loads overlap the selection.
-// SW kernels (bf16, d = 128, C a multiple of 16) stage the groups through the
-// swizzled tensor maps of `maps` (the maps of this launch's level) and accumulate
-// values on the tensor cores; the others use plain bulk copies and fp32 FMAs.
+// One select/attend pass: every level of a unit in one kernel.  A unit (query, KV
+// head) is one cluster of SPL CTAs that walks the levels top-down:
+//   level l >= 1: score + RoPE + TopK + summaries; the CTAs' parts of S^(l) are
+//                 in place for level l-1 after a cluster barrier;
+//   level 0:      score + softmax partial over A^(0);
+// then a cluster barrier and the log-sum-exp merge of every partial of the unit,
+// each CTA writing a slice of the G output heads.  Units never wait on each
+// other, so a unit's next level starts as soon as its own selection is done, and
+// the code of the scoring, selection and value loops serves all levels.
+// Each warp takes every kWarps-th parent group of its CTA's chunk; its K blocks
+// and then its V blocks stream through its ring (block numbering continues
+// across levels, so the mbarrier phases do too), so V loads overlap the
+// selection.  SW kernels (bf16, d = 128, C a multiple of 16) stage the groups
+// through the swizzled tensor maps of each level and accumulate values on the
+// tensor cores; the others use plain bulk copies and fp32 FMAs.
+// CTAs past the units' clusters (blockIdx.y >= units, decode only) re-pool the
+// ancestors of each sequence's newest token; nothing in the pass reads them.
 // ----------------------------------------------------------------------------
-template <typename T, int D, int G, bool L0, bool SW>
+constexpr int kMapLevels = 8;   // levels whose tensor maps a launch carries
+struct PassMaps {
+    KVMaps m[kMapLevels];
+};
+
+template <typename T, int D, int G, bool SW>
 __global__ void __launch_bounds__(kThreads, 2)
-    level_kernel(TreeView tv, WorkView wv, QueryView qv, const __grid_constant__ KVMaps maps,
-                 int level, int CH, int NA, int nsw) {
+    pass_kernel(TreeView tv, WorkView wv, QueryView qv, const __grid_constant__ PassMaps maps,
+                int CH, int NA, int nsw) {
     static_assert(!SW || kSwzCapable<T, D>, "swizzled staging is bf16, d = 128 only");
     extern __shared__ __align__(1024) unsigned char smem[];
-    if constexpr (L0) {
-        // CTAs past the attention grid re-pool the ancestors of each sequence's newest
-        // token (one CTA per sequence and KV head); nothing here reads them
-        const int units = qv.nq * tv.Hkv;
-        if ((int)blockIdx.y >= units) {
-            const int ci = ((int)blockIdx.y - units) * (int)gridDim.x + (int)blockIdx.x;
-            if (ci >= tv.B * tv.Hkv) return;
-            double* alpha = reinterpret_cast<double*>(smem);
-            double* pre = alpha + RECSA_MAX_C * RECSA_MAX_C;
-            for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
-            pdl_wait();
-            const int b = ci / tv.Hkv, h = ci % tv.Hkv;
-            const int64_t t = wv.lens[b] - 1;
-            __syncthreads();
-            if (t >= 1) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha);
-            return;
-        }
+    const int units = qv.nq * tv.Hkv;
+    if ((int)blockIdx.y >= units) {
+        const int ci = ((int)blockIdx.y - units) * (int)gridDim.x + (int)blockIdx.x;
+        if (ci >= tv.B * tv.Hkv) return;
+        double* alpha = reinterpret_cast<double*>(smem);
+        double* pre = alpha + RECSA_MAX_C * RECSA_MAX_C;
+        for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
+        pdl_wait();
+        const int b = ci / tv.Hkv, h = ci % tv.Hkv;
+        const int64_t t = wv.lens[b] - 1;
+        __syncthreads();
+        if (t >= 1) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha);
+        return;
     }
     constexpr int kRow = D * (int)sizeof(T);
     constexpr int V2 = VecOf<T>::N / 2;
     const int k = tv.k, C = tv.C, lgC = tv.lgC, K1 = k - 1, NL = wv.NL;
-    const int nsplit = L0 ? wv.NS0 : wv.SPL;
+    const int nsplit = wv.SPL;   // == NS0
     const int slot_bytes = C * kRow;
-    const int gsw = L0 ? 0 : gs_words(nsplit);
-    const Smem SL = smem_layout(G, D, CH, k, C, L0 ? 0 : NA, gsw, kWarps * nsw * slot_bytes);
+    const int gsw = gs_words(nsplit);
+    const Smem SL = smem_layout(G, D, CH, k, C, NA, gsw, kWarps * nsw * slot_bytes);
     float* qsm = reinterpret_cast<float*>(smem + SL.qsm);
     float4* rc4 = reinterpret_cast<float4*>(smem + SL.rc4);
-
     float* s = reinterpret_cast<float*>(smem + SL.s);
     uint32_t* key = reinterpret_cast<uint32_t*>(smem + SL.key);
     int* nodes = reinterpret_cast<int*>(smem + SL.nodes);
@@ -1265,7 +1275,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int* misc = reinterpret_cast<int*>(smem + SL.misc);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bars);
     unsigned char* ring = smem + SL.ring;
-    float* red = reinterpret_cast<float*>(smem + SL.red);   // reuses the ring after the last block
+    float* red = reinterpret_cast<float*>(smem + SL.red);   // reuses the ring between levels
     float* fm = reinterpret_cast<float*>(misc + kMiscFloat);
     if constexpr (SW) {
         // the swizzle pattern assumes 1024-byte aligned slots; every CTA of the launch
@@ -1282,43 +1292,66 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int qloc = unit / tv.Hkv, kvh = unit % tv.Hkv;
     const int gq = qv.q_begin + qloc;
     const int b = gq / qv.n_per_b;
-    // inputs no earlier kernel of the step writes: the query heads and the child
-    // rotations (staged while the previous kernel may still be finishing)
+    cg::cluster_group cluster = cg::this_cluster();
+    const int csize = (int)cluster.num_blocks();
+    const int crank = (int)cluster.block_rank();
+    // inputs no earlier kernel writes: the query heads and the child rotations
+    // (staged while the previous kernel may still be finishing)
     const T* qrow = reinterpret_cast<const T*>(qv.q) + ((int64_t)gq * tv.Hq + kvh * G) * D;
     stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
     if (threadIdx.x < kWarps * nsw) mbar_init(&bars[threadIdx.x], 1);
     mbar_fence_init();
+    if (threadIdx.x == 0) {
+        // while the kernel before (an append) may still run, this CTA's share of the
+        // RoPE table and, in a decode, its chunk of the first scored level go
+        // towards L2: those rows do not change in an append, only the list length
+        // may grow by one, so a length read before the wait is enough of a hint
+        // (the range is clamped to the tables)
+        const int nct = (int)(gridDim.x * units);
+        const int ci = unit * (int)gridDim.x + split;
+        const int per = (wv.ck + nct - 1) / nct;
+        const int r0 = ci * per, r1 = min(wv.ck, r0 + per);
+        if (r1 > r0)
+            prefetch_l2(wv.rope + (int64_t)r0 * (D / 2), (uint32_t)(r1 - r0) * (D / 2) * sizeof(float2));
+        if (qv.mode == 0) {
+            const int64_t th = *reinterpret_cast<const volatile int64_t*>(wv.lens + b);
+            const int lh = th >= 1 ? first_scored_level(th, C, lgC, k) : 0;
+            if (lh >= 1) {
+                const int nAh = list_size(th, lh, lh, C, lgC, k);
+                const int ch = ((cdiv(nAh + C - 1, C, lgC) + nsplit - 1) / nsplit) * C;
+                const int a = split * ch;
+                const int e = (int)imin64(imin64(nAh, a + ch + C), tv.rows[lh]);
+                if (e > a) {
+                    prefetch_l2(level_k<T>(tv, lh, b, kvh) + (int64_t)a * D, (uint32_t)(e - a) * kRow);
+                    prefetch_l2(level_v<T>(tv, lh, b, kvh) + (int64_t)a * D, (uint32_t)(e - a) * kRow);
+                }
+            }
+        }
+    }
     pdl_wait();
     const int64_t len = wv.lens[b];
-    if (L0 ? NL >= 1 : level < NL) {   // the parent list S^(level+1)
-        const int32_t* src = wv.sel + ((int64_t)unit * NL + level) * k;
-        for (int i = threadIdx.x; i < k; i += kThreads) par[i] = src[i];
-    }
     const int64_t t = (qv.mode == 0) ? len - 1 : qv.pos0 + (gq - b * qv.n_per_b);
     const bool valid = t >= 0 && t < len;
     const int lstar = valid ? first_scored_level(t, C, lgC, k) : 0;
     int32_t* cnt_ws = wv.cnt + (int64_t)unit * (NL + 1);
     int32_t* cnt_usr = qv.cnt_out ? qv.cnt_out + ((int64_t)gq * tv.Hkv + kvh) * (NL + 1) : nullptr;
     float* part = wv.part + (int64_t)unit * wv.NSLOT * G * (D + 2);
+    T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
     __syncthreads();
 
-    if (!L0 && (!valid || level > lstar)) {
-        // not scored for this query: its whole list is selected
+    if (!valid) {
+        // nothing to attend (empty sequence, or a prefill row beyond the length):
+        // every level unscored, a zero output
         if (split == 0) {
-            if (qv.sel_out)
-                for (int i = threadIdx.x; i < k; i += kThreads)
-                    qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k + i] = -1;
-            if (threadIdx.x == 0) {
-                cnt_ws[level] = 0;
-                if (cnt_usr) cnt_usr[level] = 0;
+            for (int l = 1; l <= NL; ++l) {
+                if (qv.sel_out)
+                    for (int i = threadIdx.x; i < k; i += kThreads)
+                        qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (l - 1)) * k + i] = -1;
+                if (threadIdx.x == 0) {
+                    cnt_ws[l] = 0;
+                    if (cnt_usr) cnt_usr[l] = 0;
+                }
             }
-        }
-        return;
-    }
-    if (L0 && !valid) {
-        // nothing to attend (empty sequence, or a prefill row beyond the length)
-        if (split == 0) {
-            T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
             for (int i = threadIdx.x; i < G * D; i += kThreads) out[i] = store_round_f<T>(0.f);
             if (threadIdx.x == 0) {
                 cnt_ws[0] = 0;
@@ -1326,255 +1359,269 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (qv.mode == 1) set_status(wv.status, kStatusBadQuery);
             }
         }
+        pdl_launch_dependents();
         return;
     }
 
-    const int nA = list_size(t, lstar, level, C, lgC, k);
-    const bool identity = (level == lstar) || (L0 && lstar == 0);
-    const int npar_all = cdiv(nA + C - 1, C, lgC);
-    const int chunk = ((npar_all + nsplit - 1) / nsplit) * C;
-    const int j0 = split * chunk;
-    const int j1 = min(nA, j0 + chunk);
-    const T *kbase, *vbase;
-    int64_t rs;
-    if (L0) {
-        kbase = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
-        vbase = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
-        rs = tv.s_t;
-    } else {
-        kbase = level_k<T>(tv, level, b, kvh);
-        vbase = level_v<T>(tv, level, b, kvh);
-        rs = D;
-    }
-    const int p_q = nA - 1;
-    // scored entries: all of A^(0); at levels >= 1 all but the current entry nA-1
-    const int n_sc = L0 ? max(0, j1 - j0) : max(0, min(j1, nA - 1) - j0);
-    if (!L0 && split == 0 && threadIdx.x == 0) {
-        cnt_ws[level] = nA;
-        if (cnt_usr) cnt_usr[level] = nA;
-    }
-    int32_t* sel_ws = L0 ? nullptr : wv.sel + ((int64_t)unit * NL + (level - 1)) * k;
-    int32_t* sel_usr = (L0 || !qv.sel_out)
-                           ? nullptr
-                           : qv.sel_out + (((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k;
-    float* outp = part + (int64_t)((L0 ? NL * wv.SPL : (level - 1) * wv.SPL) + split) * G * (D + 2);
-    if (!L0 && nA <= k) {
-        // everything selected, no summaries (not reachable below the first scored
-        // level when k, C >= 2; kept for completeness)
-        if (split == 0) {
-            for (int i = threadIdx.x; i < k; i += kThreads) {
-                int v = -1;
-                if (i < nA) v = identity ? i : C * par[cdiv(i, C, lgC)] + cmod(i, C, lgC);
-                if (i < nA) sel_ws[i] = v;
-                if (sel_usr) sel_usr[i] = v;
-            }
-        }
-        write_empty_partial(outp, G, D);
-        return;
-    }
-
-    // ---- the warp's parent groups and their blocks (K then V) ----
-    const int P = (j1 > j0) ? cdiv(j1 - j0 + C - 1, C, lgC) : 0;
-    const int nw = warp < P ? (P - warp + kWarps - 1) / kWarps : 0;
-    // logits already computed for this level (tensor-core prefill): no K blocks
-    const bool pre = !L0 && qv.pre != nullptr && level == qv.pre_level && level == lstar;
-    const int nk = pre ? 0 : nw;   // blocks [0, nk) are K, [nk, nk + nw) are V
-    const WarpRing R{ring + (size_t)warp * nsw * slot_bytes, bars + warp * nsw, nsw, slot_bytes,
-                     wv.status};
-    auto group_first = [&](int jb) -> int64_t {
-        return identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
-    };
-    auto issue = [&](int q) {
-        const int i = q < nk ? q : q - nk;
-        const int jb = j0 + (warp + kWarps * i) * C;
-        if constexpr (SW)
-            ring_issue_map(R, q, q < nk ? &maps.k : &maps.v, group_first(jb), kvh, b, C);
-        else
-            ring_issue<T, D>(R, q, q < nk ? kbase : vbase, rs, group_first(jb), min(C, j1 - jb));
-    };
-    if (identity && rs == D && threadIdx.x == 0 && j1 > j0) {
-        // the first scored level was not prefetched by a level above: its chunk
-        // (contiguous rows j0..j1) goes to L2 ahead of the ring
-        prefetch_l2(kbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
-        prefetch_l2(vbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
-    }
-    if (lane == 0)
-        for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
-    if (!L0) {
-        // the selection's histograms and published counts start at zero in every CTA
-        // of the cluster before any CTA adds into them (waited on after the scores)
-        for (int i = threadIdx.x; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
-        for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
-        if (threadIdx.x == 0) misc[kMiscPubC] = misc[kMiscPubA] = 0;
-        __syncthreads();
-        cluster_arrive();
-    }
-
-    // 1. scores of the chunk
-    if (pre) {
-        // the query's list is [0..a_t] (identity): entry j is node j
-        const float* prow = qv.pre + (int64_t)(qloc * tv.Hkv + kvh) * G * qv.pre_stride;
-        for (int i = 0; i < nw; ++i) {
-            const int jb = j0 + (warp + kWarps * i) * C;
-            const int nch = min(C, j0 + n_sc - jb);
-            for (int c = lane; c < nch; c += 32) {
-                const int r = jb - j0 + c;
-                float imp = 0.f;
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float v = __ldcg(prow + (int64_t)g * qv.pre_stride + jb + c);
-                    s[g * CH + r] = v;
-                    imp += v;
+    int qbase = 0;   // blocks this warp has taken from its ring so far
+    for (int level = NL; level >= 0; --level) {
+        const bool L0 = level == 0;
+        if (level > lstar) {
+            // not scored for this query: its whole list is selected
+            if (split == 0) {
+                if (qv.sel_out)
+                    for (int i = threadIdx.x; i < k; i += kThreads)
+                        qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k + i] = -1;
+                if (threadIdx.x == 0) {
+                    cnt_ws[level] = 0;
+                    if (cnt_usr) cnt_usr[level] = 0;
                 }
-                nodes[r] = jb + c;
-                key[r] = ordered_key(imp * (1.0f / G));
             }
+            continue;
         }
-        __syncwarp();
-    } else {
-        for (int i = 0; i < nw; ++i) {
-            const unsigned char* blk = ring_wait(R, i);
-            const int jb = j0 + (warp + kWarps * i) * C;
-            const int nch = min(C, j0 + n_sc - jb);
-            const int next_jb = (i + 1 < nw) ? jb + kWarps * C : -1;
-            if (nch > 0)
-                score_parent<T, D, G, !L0, SW>(blk, C, jb, next_jb, j0, nch, group_first(jb),
-                                               wv.rope, p_q, rc4, qsm, tv.scale, s, key, nodes,
-                                               CH);
-            __syncwarp();
-            if (lane == 0 && i + nsw < nk + nw) issue(i + nsw);
+        if (level < lstar) {
+            // the parent list S^(level+1), written by this cluster's CTAs: after the
+            // barrier every part is in place, and every CTA is past the level above
+            cluster.sync();
+            const int32_t* src = wv.sel + ((int64_t)unit * NL + level) * k;
+            for (int i = threadIdx.x; i < k; i += kThreads) par[i] = __ldcg(src + i);
         }
-    }
-    for (int i = threadIdx.x; i < n_sc; i += kThreads) flag[i] = 0;
-    // every warp's scores are written before any thread reads the chunk's (at
-    // levels >= 1 the cluster barrier below orders them)
-    if (L0) __syncthreads();
-
-    if (!L0) {
-        cg::cluster_group cluster = cg::this_cluster();
-        const int csize = (int)cluster.num_blocks();
-        const int crank = (int)cluster.block_rank();
-        const int M = nA - 1;
-        cluster_wait();   // every CTA's zeroed histograms (and, later, keys) are in place
-        __syncthreads();
-        // 2. exact top-(k-1) over all M keys; this CTA writes S for its entries
-        auto mark = [&](int i, int r) {
-            const int node = nodes[i - j0];
-            sel_ws[r] = node;
-            if (sel_usr) sel_usr[r] = node;
-            flag[i - j0] = 1;
-        };
-        bool done = true;
-        if (K1 > 0) {   // k = 1: only the current node is selected
-            uint2* pub = reinterpret_cast<uint2*>(mkey);
-            done = cluster_select(key, n_sc, j0, K1, csize, crank, gsw, hist, gs, pub,
-                                  pub + kSelCand, misc, mark);
+        if (L0) pdl_launch_dependents();   // the next kernel may start launching
+        const int nA = list_size(t, lstar, level, C, lgC, k);
+        const bool identity = level == lstar;
+        const int npar_all = cdiv(nA + C - 1, C, lgC);
+        const int chunk = ((npar_all + nsplit - 1) / nsplit) * C;
+        const int j0 = split * chunk;
+        const int j1 = min(nA, j0 + chunk);
+        const T *kbase, *vbase;
+        int64_t rs;
+        if (L0) {
+            kbase = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
+            vbase = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
+            rs = tv.s_t;
         } else {
+            kbase = level_k<T>(tv, level, b, kvh);
+            vbase = level_v<T>(tv, level, b, kvh);
+            rs = D;
+        }
+        const int p_q = nA - 1;
+        // scored entries: all of A^(0); at levels >= 1 all but the current entry nA-1
+        const int n_sc = L0 ? max(0, j1 - j0) : max(0, min(j1, nA - 1) - j0);
+        if (split == 0 && threadIdx.x == 0) {
+            cnt_ws[level] = nA;
+            if (cnt_usr) cnt_usr[level] = nA;
+        }
+        int32_t* sel_ws = L0 ? nullptr : wv.sel + ((int64_t)unit * NL + (level - 1)) * k;
+        int32_t* sel_usr = (L0 || !qv.sel_out)
+                               ? nullptr
+                               : qv.sel_out + (((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k;
+        float* outp = part + (int64_t)((L0 ? NL * wv.SPL : (level - 1) * wv.SPL) + split) * G * (D + 2);
+        if (!L0 && nA <= k) {
+            // everything selected, no summaries (not reachable below the first scored
+            // level when k, C >= 2; kept for completeness)
+            if (split == 0) {
+                for (int i = threadIdx.x; i < k; i += kThreads) {
+                    int v = -1;
+                    if (i < nA) v = identity ? i : C * par[cdiv(i, C, lgC)] + cmod(i, C, lgC);
+                    if (i < nA) sel_ws[i] = v;
+                    if (sel_usr) sel_usr[i] = v;
+                }
+            }
+            write_empty_partial(outp, G, D);
+            __syncthreads();
+            continue;
+        }
+
+        // ---- the warp's parent groups and their blocks (K then V) ----
+        const int P = (j1 > j0) ? cdiv(j1 - j0 + C - 1, C, lgC) : 0;
+        const int nw = warp < P ? (P - warp + kWarps - 1) / kWarps : 0;
+        // logits already computed for this level (tensor-core prefill): no K blocks
+        const bool pre = !L0 && qv.pre != nullptr && level == qv.pre_level && identity;
+        const int nk = pre ? 0 : nw;   // blocks [0, nk) are K, [nk, nk + nw) are V
+        const WarpRing R{ring + (size_t)warp * nsw * slot_bytes, bars + warp * nsw, nsw,
+                         slot_bytes, wv.status};
+        auto group_first = [&](int jb) -> int64_t {
+            return identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
+        };
+        const KVMaps* lmap = &maps.m[level < kMapLevels ? level : 0];
+        auto issue = [&](int q) {
+            const int i = q < nk ? q : q - nk;
+            const int jb = j0 + (warp + kWarps * i) * C;
+            if constexpr (SW)
+                ring_issue_map(R, qbase + q, q < nk ? &lmap->k : &lmap->v, group_first(jb), kvh, b, C);
+            else
+                ring_issue<T, D>(R, qbase + q, q < nk ? kbase : vbase, rs, group_first(jb),
+                                 min(C, j1 - jb));
+        };
+        if (identity && rs == D && threadIdx.x == 0 && j1 > j0) {
+            // the first scored level was not prefetched by a level above: its chunk
+            // (contiguous rows j0..j1) goes to L2 ahead of the ring
+            prefetch_l2(kbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
+            prefetch_l2(vbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
+        }
+        if (lane == 0)
+            for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
+        if (!L0) {
+            // the selection's histograms and published counts start at zero in every
+            // CTA of the cluster before any CTA adds into them (waited on after the
+            // scores)
+            for (int i = threadIdx.x; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
+            for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
+            if (threadIdx.x == 0) misc[kMiscPubC] = misc[kMiscPubA] = 0;
+            __syncthreads();
             cluster_arrive();
         }
-        if (!done) {
-            // heavy ties: every CTA's keys in list order (list position = merged
-            // index), then the block-wide select (same set)
-            for (int r = 0; r < csize; ++r) {
-                const int lo = r * chunk, hi = min(M, lo + chunk);
-                if (hi <= lo) break;
-                const uint32_t* rk = cluster.map_shared_rank(key, r);
-#pragma unroll 4
-                for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
+
+        // 1. scores of the chunk
+        if (pre) {
+            // the query's list is [0..a_t] (identity): entry j is node j
+            const float* prow = qv.pre + (int64_t)(qloc * tv.Hkv + kvh) * G * qv.pre_stride;
+            for (int i = 0; i < nw; ++i) {
+                const int jb = j0 + (warp + kWarps * i) * C;
+                const int nch = min(C, j0 + n_sc - jb);
+                for (int c = lane; c < nch; c += 32) {
+                    const int r = jb - j0 + c;
+                    float imp = 0.f;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float v = __ldcg(prow + (int64_t)g * qv.pre_stride + jb + c);
+                        s[g * CH + r] = v;
+                        imp += v;
+                    }
+                    nodes[r] = jb + c;
+                    key[r] = ordered_key(imp * (1.0f / G));
+                }
             }
-            cluster_arrive();   // remote reads done; matched by cluster_wait() before exit
-            __syncthreads();
-            select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, mark);
-        }
-        const T* nk;
-        const T* nv;
-        int64_t nrs;
-        if (level == 1) {
-            nk = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
-            nv = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
-            nrs = tv.s_t;
+            __syncwarp();
         } else {
-            nk = level_k<T>(tv, level - 1, b, kvh);
-            nv = level_v<T>(tv, level - 1, b, kvh);
-            nrs = D;
+            for (int i = 0; i < nw; ++i) {
+                const unsigned char* blk = ring_wait(R, qbase + i);
+                const int jb = j0 + (warp + kWarps * i) * C;
+                const int nch = min(C, j0 + n_sc - jb);
+                const int next_jb = (i + 1 < nw) ? jb + kWarps * C : -1;
+                if (nch > 0)
+                    score_parent<T, D, G, true, SW>(blk, C, jb, next_jb, j0, nch, group_first(jb),
+                                                    wv.rope, p_q, rc4, qsm, tv.scale, s, key,
+                                                    nodes, CH);
+                __syncwarp();
+                if (lane == 0 && i + nsw < nk + nw) issue(i + nsw);
+            }
         }
-        if (crank == 0 && threadIdx.x == 0) {
-            const int64_t cur = apow(t, level, C, lgC);
-            sel_ws[K1] = (int)cur;
-            if (sel_usr) sel_usr[K1] = (int)cur;
-            prefetch_children<T, D>(nk, nv, nrs, (int64_t)C * cur,
-                                    (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1));
-        }
+        for (int i = threadIdx.x; i < n_sc; i += kThreads) flag[i] = 0;
         __syncthreads();
-        // the children of this chunk's selected nodes are the next level's rows: to L2,
-        // each thread for its own entries, so the requests go out in parallel
-        for (int i = threadIdx.x; i < n_sc; i += kThreads)
-            if (flag[i]) prefetch_children<T, D>(nk, nv, nrs, (int64_t)C * nodes[i], C);
+
+        if (!L0) {
+            const int M = nA - 1;
+            cluster_wait();   // every CTA's zeroed histograms (and keys) are in place
+            // 2. exact top-(k-1) over all M keys; this CTA writes S for its entries
+            auto mark = [&](int i, int r) {
+                const int node = nodes[i - j0];
+                sel_ws[r] = node;
+                if (sel_usr) sel_usr[r] = node;
+                flag[i - j0] = 1;
+            };
+            bool done = true;
+            if (K1 > 0) {   // k = 1: only the current node is selected
+                uint2* pub = reinterpret_cast<uint2*>(mkey);
+                done = cluster_select(key, n_sc, j0, K1, csize, crank, gsw, hist, gs, pub,
+                                      pub + kSelCand, misc, mark);
+            } else {
+                cluster_arrive();
+            }
+            if (!done) {
+                // heavy ties: every CTA's keys in list order (list position = merged
+                // index), then the block-wide select (same set)
+                for (int r = 0; r < csize; ++r) {
+                    const int lo = r * chunk, hi = min(M, lo + chunk);
+                    if (hi <= lo) break;
+                    const uint32_t* rk = cluster.map_shared_rank(key, r);
+#pragma unroll 4
+                    for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
+                }
+                cluster_arrive();   // remote reads done; matched by cluster_wait() below
+                __syncthreads();
+                select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, mark);
+            }
+            const T* nk_;
+            const T* nv_;
+            int64_t nrs;
+            if (level == 1) {
+                nk_ = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
+                nv_ = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
+                nrs = tv.s_t;
+            } else {
+                nk_ = level_k<T>(tv, level - 1, b, kvh);
+                nv_ = level_v<T>(tv, level - 1, b, kvh);
+                nrs = D;
+            }
+            if (crank == 0 && threadIdx.x == 0) {
+                const int64_t cur = apow(t, level, C, lgC);
+                sel_ws[K1] = (int)cur;
+                if (sel_usr) sel_usr[K1] = (int)cur;
+                prefetch_children<T, D>(nk_, nv_, nrs, (int64_t)C * cur,
+                                        (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1));
+            }
+            __syncthreads();
+            // the children of this chunk's selected nodes are the next level's rows: to
+            // L2, each thread for its own entries, so the requests go out in parallel
+            for (int i = threadIdx.x; i < n_sc; i += kThreads)
+                if (flag[i]) prefetch_children<T, D>(nk_, nv_, nrs, (int64_t)C * nodes[i], C);
+        }
+
+        // 3. softmax partial over the unselected (level) or all (level 0) entries
+        float lsum[G];
+        // (scratch: the histogram area; the ring, and so red, still holds V blocks)
+        softmax_weights<G>(s, n_sc, L0 ? nullptr : flag, CH, reinterpret_cast<float*>(hist), fm,
+                           lsum);
+        if constexpr (SW) {
+            float acc[D / 16][4];
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+            for (int i = 0; i < nw; ++i) {
+                const int q = nk + i;
+                const unsigned char* blk = ring_wait(R, qbase + q);
+                const int jb = j0 + (warp + kWarps * i) * C;
+                const int nrow = min(C, j0 + n_sc - jb);
+                if (nrow > 0 && fm[0] > -INFINITY)
+                    accum_parent_mma<D, G>(blk, C, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
+                __syncwarp();
+                if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
+            }
+            __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
+            finish_partial_mma<D, G>(acc, lsum, fm, red, outp);
+        } else {
+            float2 acc[G][V2];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < V2; ++e) acc[g][e] = make_float2(0.f, 0.f);
+            for (int i = 0; i < nw; ++i) {
+                const int q = nk + i;
+                const unsigned char* blk = ring_wait(R, qbase + q);
+                const int jb = j0 + (warp + kWarps * i) * C;
+                const int nrow = min(C, j0 + n_sc - jb);
+                if (nrow > 0 && fm[0] > -INFINITY)
+                    accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
+                __syncwarp();
+                if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
+            }
+            __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
+            finish_partial<T, D, G>(acc, lsum, fm, red, outp);
+        }
+        qbase += nk + nw;
+        // red (the ring) is read: the next level's tensor copies may overwrite it
+        __syncthreads();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!L0) cluster_wait();   // matches the arrive after this CTA's remote reads
     }
 
-    // the next kernel may start launching: what remains here is this CTA's partial
-    pdl_launch_dependents();
-    // 4. softmax partial over the unselected (level) or all (level 0) entries
-    float lsum[G];
-    // (scratch: the histogram area; the ring, and so red, still holds V blocks)
-    softmax_weights<G>(s, n_sc, L0 ? nullptr : flag, CH, reinterpret_cast<float*>(hist), fm, lsum);
-    if constexpr (SW) {
-        float acc[D / 16][4];
-#pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-        for (int i = 0; i < nw; ++i) {
-            const int q = nk + i;
-            const unsigned char* blk = ring_wait(R, q);
-            const int jb = j0 + (warp + kWarps * i) * C;
-            const int nrow = min(C, j0 + n_sc - jb);
-            if (nrow > 0 && fm[0] > -INFINITY)
-                accum_parent_mma<D, G>(blk, C, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
-            __syncwarp();
-            if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
-        }
-        __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
-        finish_partial_mma<D, G>(acc, lsum, fm, red, outp);
-    } else {
-        float2 acc[G][V2];
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < V2; ++e) acc[g][e] = make_float2(0.f, 0.f);
-        for (int i = 0; i < nw; ++i) {
-            const int q = nk + i;
-            const unsigned char* blk = ring_wait(R, q);
-            const int jb = j0 + (warp + kWarps * i) * C;
-            const int nrow = min(C, j0 + n_sc - jb);
-            if (nrow > 0 && fm[0] > -INFINITY)
-                accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
-            __syncwarp();
-            if (lane == 0 && q + nsw < nk + nw) issue(q + nsw);
-        }
-        __syncthreads();   // every block consumed: the ring area becomes the reduction buffer
-        finish_partial<T, D, G>(acc, lsum, fm, red, outp);
-    }
-
-    if (L0) {
-        if (split == 0 && threadIdx.x == 0) {
-            cnt_ws[0] = nA;
-            if (cnt_usr) cnt_usr[0] = nA;
-        }
-        // the last CTA of this unit to finish merges all of the unit's partials
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0)
-            misc[kMiscLast] = (atomicAdd(&wv.ucnt[unit], 1u) == (unsigned)nsplit - 1) ? 1 : 0;
-        __syncthreads();
-        if (misc[kMiscLast]) {
-            __threadfence();
-            T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
-            combine_unit<T, D, G>(part, lstar, wv.SPL, wv.NS0, NL, out, red,
-                                  reinterpret_cast<float*>(misc + kMiscFloat + 8));
-            if (threadIdx.x == 0) wv.ucnt[unit] = 0u;
-        }
-    } else {
-        cluster_wait();
-    }
+    // every partial of the unit is written: merge them, this CTA taking a slice of
+    // the G output heads
+    cluster.sync();
+    const int per = (G * D + csize - 1) / csize;
+    combine_unit<T, D, G>(part, lstar, wv.SPL, wv.NS0, NL, out, red,
+                          reinterpret_cast<float*>(misc + kMiscFloat + 8), crank * per,
+                          min(G * D, (crank + 1) * per));
 }
 
 // ----------------------------------------------------------------------------
@@ -1585,39 +1632,37 @@ static inline int chunk_cap(int k, int splits, int C) { return ((k + splits - 1)
 // blocks in flight per warp: two when a parent group is at most 4 KB
 static inline int slots_per_warp(int C, int D, int esize) { return C * D * esize <= 4096 ? 2 : 1; }
 
+// Shared memory of the pass kernel (walk CTAs included when `walk`).
 template <typename T, int D, int G>
-static size_t level_smem(int C, int k, int splits, bool l0) {
+static size_t pass_smem(int C, int k, int splits, int n_levels, bool walk) {
     const int CH = chunk_cap(k, splits, C);
     const int nsw = slots_per_warp(C, D, (int)sizeof(T));
-    return smem_layout(G, D, CH, k, C, l0 ? 0 : C * k, l0 ? 0 : gs_words(splits),
-                       kWarps * nsw * C * D * (int)sizeof(T))
-        .total;
+    const size_t sm = smem_layout(G, D, CH, k, C, C * k, gs_words(splits),
+                                  kWarps * nsw * C * D * (int)sizeof(T))
+                          .total;
+    const size_t ws = walk ? ancestor_walk_smem(n_levels, D) : 0;
+    return sm > ws ? sm : ws;
 }
 
 template <typename T, int D, int G, bool SW>
-static cudaError_t prepare_variant(size_t sm, size_t sm0, int SPL) {
-    cudaError_t e = cudaFuncSetAttribute(level_kernel<T, D, G, false, SW>,
+static cudaError_t prepare_variant(size_t sm, int SPL) {
+    cudaError_t e = cudaFuncSetAttribute(pass_kernel<T, D, G, SW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    if (SPL > 8) {
-        e = cudaFuncSetAttribute(level_kernel<T, D, G, false, SW>,
+    if (SPL > 8)
+        e = cudaFuncSetAttribute(pass_kernel<T, D, G, SW>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
-    const size_t walk = ancestor_walk_smem(kMaxLevels, D);
-    return cudaFuncSetAttribute(level_kernel<T, D, G, true, SW>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(sm0 > walk ? sm0 : walk));
+    return e;
 }
 
 template <typename T, int D, int G>
 static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
-    const size_t sm = level_smem<T, D, G>(C, k, SPL, false);
-    const size_t sm0 = level_smem<T, D, G>(C, k, NS0, true);
-    if (sm > 227 * 1024 || sm0 > 227 * 1024) return cudaErrorInvalidValue;
-    cudaError_t e = prepare_variant<T, D, G, false>(sm, sm0, SPL);
+    if (NS0 != SPL) return cudaErrorInvalidValue;   // level 0 runs on the same cluster
+    const size_t sm = pass_smem<T, D, G>(C, k, SPL, kMaxLevels, true);
+    if (sm > 227 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = prepare_variant<T, D, G, false>(sm, SPL);
     if constexpr (kSwzCapable<T, D>)
-        if (e == cudaSuccess) e = prepare_variant<T, D, G, true>(sm, sm0, SPL);
+        if (e == cudaSuccess) e = prepare_variant<T, D, G, true>(sm, SPL);
     return e;
 }
 
@@ -1625,65 +1670,44 @@ template <typename T, int D, int G, bool SW>
 static cudaError_t select_attend_variant(const TreeView& tv, const WorkView& wv,
                                          const QueryView& qv, cudaStream_t s, const ProfHook* prof,
                                          const KVMaps* maps) {
-    static const KVMaps kNoMaps = {};
-    const int CH = chunk_cap(tv.k, wv.SPL, tv.C), CH0 = chunk_cap(tv.k, wv.NS0, tv.C);
+    PassMaps pm = {};
+    if (SW)
+        for (int l = 0; l < tv.n_levels && l < kMapLevels; ++l) pm.m[l] = maps[l];
+    const int CH = chunk_cap(tv.k, wv.SPL, tv.C);
     const int NA = tv.C * tv.k;
     const int nsw = slots_per_warp(tv.C, D, (int)sizeof(T));
-    const size_t sm = level_smem<T, D, G>(tv.C, tv.k, wv.SPL, false);
-    const size_t sm0 = level_smem<T, D, G>(tv.C, tv.k, wv.NS0, true);
     const unsigned units = (unsigned)(qv.nq * tv.Hkv);
-    for (int level = wv.NL; level >= 1; --level) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)wv.SPL, units, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = sm;
-        cfg.stream = s;
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)wv.SPL;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        attr[1] = pdl_attribute();
-        cfg.attrs = attr;
-        cfg.numAttrs = 2;
-        prof_mark(prof, level, true, s);
-        cudaError_t e = cudaLaunchKernelEx(&cfg, level_kernel<T, D, G, false, SW>, tv, wv, qv,
-                                           SW ? maps[level] : kNoMaps, level, CH, NA, nsw);
-        prof_mark(prof, level, false, s);
-        if (e != cudaSuccess) return e;
-    }
-    cudaLaunchConfig_t cfg0 = {};
     // with a pending ancestor walk, extra rows of CTAs (one CTA per sequence and KV head)
-    const unsigned walk_rows =
-        qv.walk ? (unsigned)((tv.B * tv.Hkv + wv.NS0 - 1) / wv.NS0) : 0u;
-    const size_t walk_sm = ancestor_walk_smem(tv.n_levels, D);
-    cfg0.gridDim = dim3((unsigned)wv.NS0, units + walk_rows, 1);
-    cfg0.blockDim = dim3(kThreads, 1, 1);
-    cfg0.dynamicSmemBytes = (qv.walk && walk_sm > sm0) ? walk_sm : sm0;
-    cfg0.stream = s;
-    cudaLaunchAttribute attr0[1] = {pdl_attribute()};
-    cfg0.attrs = attr0;
-    cfg0.numAttrs = 1;
+    const unsigned walk_rows = qv.walk ? (unsigned)((tv.B * tv.Hkv + wv.SPL - 1) / wv.SPL) : 0u;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)wv.SPL, units + walk_rows, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pass_smem<T, D, G>(tv.C, tv.k, wv.SPL, tv.n_levels, qv.walk != 0);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)wv.SPL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attribute();
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     prof_mark(prof, 0, true, s);
-    cudaError_t e0 = cudaLaunchKernelEx(&cfg0, level_kernel<T, D, G, true, SW>, tv, wv, qv,
-                                        SW ? maps[0] : kNoMaps, 0, CH0, 0, nsw);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pass_kernel<T, D, G, SW>, tv, wv, qv, pm, CH, NA, nsw);
     prof_mark(prof, 0, false, s);
-    if (e0 != cudaSuccess) return e0;
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 // maps: the tensor maps of every level when the tree stages through them (bf16,
-// d = 128, C a multiple of 16), else null.
+// d = 128, C a multiple of 16, at most kMapLevels levels), else null.
 template <typename T, int D, int G>
 static cudaError_t select_attend_impl(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                       cudaStream_t s, const ProfHook* prof, const KVMaps* maps) {
     if constexpr (kSwzCapable<T, D>) {
-        if (maps) {
-            if (tv.C % 16 != 0 || tv.n_levels > kMaxLevels) return cudaErrorInvalidValue;
+        if (maps && tv.C % 16 == 0 && tv.n_levels <= kMapLevels)
             return select_attend_variant<T, D, G, true>(tv, wv, qv, s, prof, maps);
-        }
     }
-    if (maps) return cudaErrorInvalidValue;
     return select_attend_variant<T, D, G, false>(tv, wv, qv, s, prof, nullptr);
 }
 
