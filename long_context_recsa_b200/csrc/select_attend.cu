@@ -117,7 +117,7 @@ constexpr int kSelCand = 384;   // candidates of the cluster selection's boundar
 // been consumed.  mkey holds the exchanged keys of the heavy-tie path, or the
 // published and gathered candidates of the cluster selection.
 __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, int NA, int gsw,
-                                            int ring_bytes) {
+                                            int nslot, int ring_bytes) {
     Smem L;
     size_t o = 0;
     L.qsm = o;   o = align16(o + sizeof(float) * G * D);
@@ -126,7 +126,7 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
     L.key = o;   o = align16(o + sizeof(uint32_t) * CH);
     L.nodes = o; o = align16(o + sizeof(int) * CH);
     L.flag = o;  o = align16(o + sizeof(unsigned char) * CH);
-    L.par = o;   o = align16(o + sizeof(int) * k);
+    L.par = o;   o = align16(o + sizeof(int) * 2 * k);   // this level's parents, the next's
     const int mk = NA > 0 && NA < 4 * kSelCand ? 4 * kSelCand : NA;
     L.mkey = o;  o = align16(o + sizeof(uint32_t) * mk);
     L.hist = o;  o = align16(o + sizeof(uint32_t) * 1024);   // >= kSelBins / 2, radix 512
@@ -136,7 +136,10 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
     o = (o + 1023) & ~size_t(1023);   // swizzled slots need 1024-byte alignment
     L.ring = o;
     L.red = o;
-    const size_t red_bytes = sizeof(float) * kWarps * G * (D + 1);
+    // the value reduction, or the merge's weights, (m, l) and one slot column
+    size_t red_bytes = sizeof(float) * kWarps * G * (D + 1);
+    const size_t merge_bytes = sizeof(float) * (size_t)(3 * G + 1) * nslot;
+    if (merge_bytes > red_bytes) red_bytes = merge_bytes;
     o += (size_t)ring_bytes > red_bytes ? (size_t)ring_bytes : red_bytes;
     L.total = o;
     return L;
@@ -665,19 +668,14 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// cnt consecutive rows starting at row `first` (row stride rs), K and V.
+// cnt consecutive rows starting at row `first` of a table with row stride rs.
 template <typename T, int D>
-__device__ __forceinline__ void prefetch_children(const T* kb, const T* vb, int64_t rs,
-                                                  int64_t first, int cnt) {
+__device__ __forceinline__ void prefetch_rows(const T* base, int64_t rs, int64_t first, int cnt) {
     constexpr uint32_t kRow = D * sizeof(T);
     if (rs == D) {
-        prefetch_l2(kb + first * D, cnt * kRow);
-        prefetch_l2(vb + first * D, cnt * kRow);
+        prefetch_l2(base + first * D, cnt * kRow);
     } else {
-        for (int c = 0; c < cnt; ++c) {
-            prefetch_l2(kb + (first + c) * rs, kRow);
-            prefetch_l2(vb + (first + c) * rs, kRow);
-        }
+        for (int c = 0; c < cnt; ++c) prefetch_l2(base + (first + c) * rs, kRow);
     }
 }
 
@@ -1167,28 +1165,37 @@ __device__ __forceinline__ void write_empty_partial(float* outp, int G, int D) {
 }
 
 // Log-sum-exp merge of a unit's partials into its G output heads, output elements
-// [e0, e1) of the G*D.  Partials of other CTAs are read through L2 (ld.global.cg).
+// [e0, e1) of the G*D.  Partials of other CTAs are read through L2 (ld.global.cg),
+// all of a slice's loads issued together into shared memory (buf, nbuf floats:
+// weights, (m, l) of every slot and head, then the staged values) so they cost one
+// latency rather than one per slot; the sums run over the slots in slot order.
 template <typename T, int D, int G>
 __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL, T* out,
-                             float* wsh /* >= G*(NL*SPL+NS0) */, float* Lsh /* G */, int e0,
-                             int e1) {
+                             float* buf, int nbuf, float* Lsh /* G */, int e0, int e1) {
     const int nls = lstar * SPL;
     const int ns = nls + NS0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* wsh = buf;            // [G][ns] weights
+    float* mm = buf + G * ns;    // [G][ns] m
+    float* ll = mm + G * ns;     // [G][ns] l
+    float* vals = ll + G * ns;   // [ns][E] staged values
+    auto slot_of = [&](int i) { return i < nls ? i : NL * SPL + (i - nls); };
+    for (int x = threadIdx.x; x < ns * G; x += kThreads) {
+        const int i = x / G, g = x % G;
+        const float* rec = P + (slot_of(i) * G + g) * (D + 2);
+        mm[g * ns + i] = __ldcg(rec + D);
+        ll[g * ns + i] = __ldcg(rec + D + 1);
+    }
+    __syncthreads();
     for (int g = warp; g < G; g += kWarps) {
         float M = -INFINITY;
-        for (int i = lane; i < ns; i += 32) {
-            const int slot = i < nls ? i : NL * SPL + (i - nls);
-            M = fmaxf(M, __ldcg(P + (slot * G + g) * (D + 2) + D));
-        }
+        for (int i = lane; i < ns; i += 32) M = fmaxf(M, mm[g * ns + i]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
         float L = 0.f;
         for (int i = lane; i < ns; i += 32) {
-            const int slot = i < nls ? i : NL * SPL + (i - nls);
-            const float m = __ldcg(P + (slot * G + g) * (D + 2) + D);
-            const float l = __ldcg(P + (slot * G + g) * (D + 2) + D + 1);
-            const float w = l > 0.f ? __expf(m - M) : 0.f;
+            const float l = ll[g * ns + i];
+            const float w = l > 0.f ? __expf(mm[g * ns + i] - M) : 0.f;
             wsh[g * ns + i] = w;
             L += w * l;
         }
@@ -1196,17 +1203,22 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
         for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
         if (lane == 0) Lsh[g] = L;
     }
-    __syncthreads();
-    for (int e = e0 + (int)threadIdx.x; e < e1; e += kThreads) {
-        const int g = e / D, d = e % D;
-        float O = 0.f;
-#pragma unroll 4
-        for (int i = 0; i < ns; ++i) {
-            const int slot = i < nls ? i : NL * SPL + (i - nls);
-            O += wsh[g * ns + i] * __ldcg(P + (slot * G + g) * (D + 2) + d);
+    const int cap = (nbuf - 3 * G * ns) / ns;   // output elements staged per round
+    for (int c0 = e0; c0 < e1; c0 += cap) {
+        const int E = min(cap, e1 - c0);
+        __syncthreads();   // the previous round's reads (and the weights) are done
+        for (int x = threadIdx.x; x < ns * E; x += kThreads) {
+            const int i = x / E, e = c0 + x % E;
+            vals[x] = __ldcg(P + (slot_of(i) * G + e / D) * (D + 2) + e % D);
         }
-        const float L = Lsh[g];
-        out[e] = store_round_f<T>(L > 0.f ? O / L : 0.f);
+        __syncthreads();
+        for (int x = threadIdx.x; x < E; x += kThreads) {
+            const int e = c0 + x, g = e / D;
+            float O = 0.f;
+            for (int i = 0; i < ns; ++i) O += wsh[g * ns + i] * vals[i * E + x];
+            const float L = Lsh[g];
+            out[e] = store_round_f<T>(L > 0.f ? O / L : 0.f);
+        }
     }
 }
 
@@ -1261,14 +1273,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nsplit = wv.SPL;   // == NS0
     const int slot_bytes = C * kRow;
     const int gsw = gs_words(nsplit);
-    const Smem SL = smem_layout(G, D, CH, k, C, NA, gsw, kWarps * nsw * slot_bytes);
+    const Smem SL = smem_layout(G, D, CH, k, C, NA, gsw, wv.NSLOT, kWarps * nsw * slot_bytes);
     float* qsm = reinterpret_cast<float*>(smem + SL.qsm);
     float4* rc4 = reinterpret_cast<float4*>(smem + SL.rc4);
     float* s = reinterpret_cast<float*>(smem + SL.s);
     uint32_t* key = reinterpret_cast<uint32_t*>(smem + SL.key);
     int* nodes = reinterpret_cast<int*>(smem + SL.nodes);
     unsigned char* flag = smem + SL.flag;
+    // par: S^(level+1), the parents of this level's list (entries this CTA needs);
+    // par_next: S^(level), filled by the cluster's CTAs as they select
     int* par = reinterpret_cast<int*>(smem + SL.par);
+    int* par_next = par + k;
     uint32_t* mkey = reinterpret_cast<uint32_t*>(smem + SL.mkey);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + SL.hist);
     uint32_t* gs = reinterpret_cast<uint32_t*>(smem + SL.gs);
@@ -1301,6 +1316,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
     if (threadIdx.x < kWarps * nsw) mbar_init(&bars[threadIdx.x], 1);
     mbar_fence_init();
+    if constexpr (SW) {
+        // the levels' tensor-map descriptors into the descriptor cache
+        if (threadIdx.x < 2 * kMapLevels && threadIdx.x / 2 <= NL) {
+            const KVMaps& m = maps.m[threadIdx.x / 2];
+            asm volatile("prefetch.tensormap [%0];" ::"l"(
+                             reinterpret_cast<uint64_t>((threadIdx.x & 1) ? &m.v : &m.k))
+                         : "memory");
+        }
+    }
     if (threadIdx.x == 0) {
         // while the kernel before (an append) may still run, this CTA's share of the
         // RoPE table and, in a decode, its chunk of the first scored level go
@@ -1366,27 +1390,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     int qbase = 0;   // blocks this warp has taken from its ring so far
     for (int level = NL; level >= 0; --level) {
         const bool L0 = level == 0;
-        if (level > lstar) {
-            // not scored for this query: its whole list is selected
-            if (split == 0) {
-                if (qv.sel_out)
-                    for (int i = threadIdx.x; i < k; i += kThreads)
-                        qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k + i] = -1;
-                if (threadIdx.x == 0) {
-                    cnt_ws[level] = 0;
-                    if (cnt_usr) cnt_usr[level] = 0;
-                }
-            }
-            continue;
-        }
+        if (level > lstar) continue;   // not scored: recorded after the pass
         if (level < lstar) {
-            // the parent list S^(level+1), written by this cluster's CTAs: after the
-            // barrier every part is in place, and every CTA is past the level above
+            // the parent list S^(level+1): every CTA of the cluster has stored the
+            // entries this CTA needs into its par_next; after the barrier they are in
+            // place, and every CTA is past the level above
             cluster.sync();
-            const int32_t* src = wv.sel + ((int64_t)unit * NL + level) * k;
-            for (int i = threadIdx.x; i < k; i += kThreads) par[i] = __ldcg(src + i);
+            int* tmp = par;
+            par = par_next;
+            par_next = tmp;
         }
-        if (L0) pdl_launch_dependents();   // the next kernel may start launching
+        if (!L0) {
+            // the selection's histograms and published counts start at zero in every
+            // CTA of the cluster before any CTA adds into them (waited on after the
+            // scores).  Done first at a level, so the release has no other stores of
+            // this CTA to wait for.
+            for (int i = threadIdx.x; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
+            for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
+            if (threadIdx.x == 0) misc[kMiscPubC] = misc[kMiscPubA] = 0;
+            __syncthreads();
+            cluster_arrive();
+        } else {
+            pdl_launch_dependents();   // the next kernel may start launching
+        }
         const int nA = list_size(t, lstar, level, C, lgC, k);
         const bool identity = level == lstar;
         const int npar_all = cdiv(nA + C - 1, C, lgC);
@@ -1416,6 +1442,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                                ? nullptr
                                : qv.sel_out + (((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k;
         float* outp = part + (int64_t)((L0 ? NL * wv.SPL : (level - 1) * wv.SPL) + split) * G * (D + 2);
+        // parents per CTA at the next level: parent rank r goes to CTA r / ppc_next
+        int ppc_next = 1;
+        if (!L0) {
+            const int nA_next = list_size(t, lstar, level - 1, C, lgC, k);
+            const int npar_next = cdiv(nA_next + C - 1, C, lgC);
+            ppc_next = (npar_next + nsplit - 1) / nsplit;
+        }
         if (!L0 && nA <= k) {
             // everything selected, no summaries (not reachable below the first scored
             // level when k, C >= 2; kept for completeness)
@@ -1423,12 +1456,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int i = threadIdx.x; i < k; i += kThreads) {
                     int v = -1;
                     if (i < nA) v = identity ? i : C * par[cdiv(i, C, lgC)] + cmod(i, C, lgC);
-                    if (i < nA) sel_ws[i] = v;
+                    if (i < nA) {
+                        sel_ws[i] = v;
+                        cluster.map_shared_rank(par_next, i / ppc_next)[i] = v;
+                    }
                     if (sel_usr) sel_usr[i] = v;
                 }
             }
             write_empty_partial(outp, G, D);
             __syncthreads();
+            cluster_wait();   // matches the arrive at the level's start
             continue;
         }
 
@@ -1461,16 +1498,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (lane == 0)
             for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
-        if (!L0) {
-            // the selection's histograms and published counts start at zero in every
-            // CTA of the cluster before any CTA adds into them (waited on after the
-            // scores)
-            for (int i = threadIdx.x; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
-            for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
-            if (threadIdx.x == 0) misc[kMiscPubC] = misc[kMiscPubA] = 0;
-            __syncthreads();
-            cluster_arrive();
-        }
 
         // 1. scores of the chunk
         if (pre) {
@@ -1519,6 +1546,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 sel_ws[r] = node;
                 if (sel_usr) sel_usr[r] = node;
                 flag[i - j0] = 1;
+                cluster.map_shared_rank(par_next, r / ppc_next)[r] = node;
             };
             bool done = true;
             if (K1 > 0) {   // k = 1: only the current node is selected
@@ -1558,14 +1586,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int64_t cur = apow(t, level, C, lgC);
                 sel_ws[K1] = (int)cur;
                 if (sel_usr) sel_usr[K1] = (int)cur;
-                prefetch_children<T, D>(nk_, nv_, nrs, (int64_t)C * cur,
-                                        (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1));
+                cluster.map_shared_rank(par_next, K1 / ppc_next)[K1] = (int)cur;
+                const int nch = (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1);
+                prefetch_rows<T, D>(nk_, nrs, (int64_t)C * cur, nch);
+                prefetch_rows<T, D>(nv_, nrs, (int64_t)C * cur, nch);
             }
             __syncthreads();
             // the children of this chunk's selected nodes are the next level's rows: to
             // L2, each thread for its own entries, so the requests go out in parallel
             for (int i = threadIdx.x; i < n_sc; i += kThreads)
-                if (flag[i]) prefetch_children<T, D>(nk_, nv_, nrs, (int64_t)C * nodes[i], C);
+                if (flag[i]) {
+                    prefetch_rows<T, D>(nk_, nrs, (int64_t)C * nodes[i], C);
+                    prefetch_rows<T, D>(nv_, nrs, (int64_t)C * nodes[i], C);
+                }
         }
 
         // 3. softmax partial over the unselected (level) or all (level 0) entries
@@ -1615,11 +1648,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!L0) cluster_wait();   // matches the arrive after this CTA's remote reads
     }
 
+    if (split == 0) {
+        // the levels above the first scored one: their whole lists are selected
+        for (int l = lstar + 1; l <= NL; ++l) {
+            if (qv.sel_out)
+                for (int i = threadIdx.x; i < k; i += kThreads)
+                    qv.sel_out[(((int64_t)gq * tv.Hkv + kvh) * NL + (l - 1)) * k + i] = -1;
+            if (threadIdx.x == 0) {
+                cnt_ws[l] = 0;
+                if (cnt_usr) cnt_usr[l] = 0;
+            }
+        }
+    }
     // every partial of the unit is written: merge them, this CTA taking a slice of
     // the G output heads
     cluster.sync();
     const int per = (G * D + csize - 1) / csize;
     combine_unit<T, D, G>(part, lstar, wv.SPL, wv.NS0, NL, out, red,
+                          (int)((SL.total - SL.red) / sizeof(float)),
                           reinterpret_cast<float*>(misc + kMiscFloat + 8), crank * per,
                           min(G * D, (crank + 1) * per));
 }
@@ -1634,10 +1680,10 @@ static inline int slots_per_warp(int C, int D, int esize) { return C * D * esize
 
 // Shared memory of the pass kernel (walk CTAs included when `walk`).
 template <typename T, int D, int G>
-static size_t pass_smem(int C, int k, int splits, int n_levels, bool walk) {
+static size_t pass_smem(int C, int k, int splits, int nslot, int n_levels, bool walk) {
     const int CH = chunk_cap(k, splits, C);
     const int nsw = slots_per_warp(C, D, (int)sizeof(T));
-    const size_t sm = smem_layout(G, D, CH, k, C, C * k, gs_words(splits),
+    const size_t sm = smem_layout(G, D, CH, k, C, C * k, gs_words(splits), nslot,
                                   kWarps * nsw * C * D * (int)sizeof(T))
                           .total;
     const size_t ws = walk ? ancestor_walk_smem(n_levels, D) : 0;
@@ -1658,7 +1704,7 @@ static cudaError_t prepare_variant(size_t sm, int SPL) {
 template <typename T, int D, int G>
 static cudaError_t prepare_impl(int SPL, int NS0, int C, int k) {
     if (NS0 != SPL) return cudaErrorInvalidValue;   // level 0 runs on the same cluster
-    const size_t sm = pass_smem<T, D, G>(C, k, SPL, kMaxLevels, true);
+    const size_t sm = pass_smem<T, D, G>(C, k, SPL, kMaxLevels * SPL + NS0, kMaxLevels, true);
     if (sm > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = prepare_variant<T, D, G, false>(sm, SPL);
     if constexpr (kSwzCapable<T, D>)
@@ -1682,7 +1728,7 @@ static cudaError_t select_attend_variant(const TreeView& tv, const WorkView& wv,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)wv.SPL, units + walk_rows, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = pass_smem<T, D, G>(tv.C, tv.k, wv.SPL, tv.n_levels, qv.walk != 0);
+    cfg.dynamicSmemBytes = pass_smem<T, D, G>(tv.C, tv.k, wv.SPL, wv.NSLOT, tv.n_levels, qv.walk != 0);
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
