@@ -66,7 +66,8 @@ def test_tiny_fp32_config(R):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("C,k,d,G", [(4, 3, 64, 2), (16, 8, 128, 4), (2, 5, 64, 1), (8, 16, 128, 8)])
+@pytest.mark.parametrize("C,k,d,G", [(4, 3, 64, 2), (16, 8, 128, 4), (2, 5, 64, 1), (8, 16, 128, 8),
+                                     (16, 8, 128, 1), (16, 4, 128, 2), (16, 8, 128, 8)])
 def test_small_ragged_batches(R, dtype, C, k, d, G):
     Hkv = 2
     lengths = [1000, 777, 64 * C + 1, 5]
