@@ -218,6 +218,50 @@ def test_long_lists_sampled_select(R, k, L):
                     dtype="bf16", cap=L, n_needles=16)
 
 
+
+def test_k512_two_selecting_levels(R):
+    """k = 512 (C*k = 8192, the largest list the library takes): L = 140000 selects
+    at level 2 (547 nodes) and at level 1 (8192 children), then attends level 0."""
+    tree, worst = run_decode_case(R, config_id=19, B=1, Hkv=2, Hq=8, d=128, C=16, k=512,
+                                  lengths=[140000], dtype="bf16", cap=140000, n_needles=16)
+    assert tree.n_sel_levels >= 2
+
+
+def test_whole_sequence_chunked_prefill(R):
+    """A whole sequence through the public calls, as a model runs it: per chunk, append
+    its K/V rows (the tree grows, starting empty), then prefill its query rows.
+    Sampled rows of every chunk (first, middle, last) against the oracle, whose rows
+    depend only on tokens <= t; the final tree bit for bit."""
+    from oracle import recsa_oracle as O_
+    C, k, d, Hkv, Hq = 16, 64, 128, 2, 8
+    L, n = 9000, 2048
+    G = Hq // Hkv
+    w = H.w_for(C)
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype="bf16", pooler_w=w)
+    K, V, Q = H.make_inputs(20, 1, Hkv, Hq, d, L, [L], "bf16", q_rows=L, n_needles=8)
+    tree = R.RecsaTree(cfg, L, 1, max_queries=256, k0=torch.zeros_like(K),
+                       v0=torch.zeros_like(V))
+    levels = [O_.build_tree(H.to64(K[0, h]), H.to64(V[0, h]), C, np.asarray(w, dtype=np.float64),
+                            "bf16") for h in range(Hkv)]
+    for p0 in range(0, L, n):
+        m = min(n, L - p0)
+        tree.recsa_append(K[:, :, p0:p0 + m].contiguous(), V[:, :, p0:p0 + m].contiguous())
+        O, sel, cnt = tree.prefill(Q[:, p0:p0 + m].contiguous(), p0, with_sel=True)
+        torch.cuda.synchronize()
+        assert tree.recsa_get_status() == R.RECSA_OK
+        assert tree.host_lengths() == [p0 + m]
+        for i in sorted({0, m // 2, m - 1}):
+            t = p0 + i
+            for h in range(Hkv):
+                qg = H.to64(Q[0, t, h * G:(h + 1) * G])
+                res = O_.select_and_attend(levels[h], qg, t, C, k, base=1e6)
+                cur = H.check_selection(levels[h], qg, t, C, k, 1e6, res, sel[i, h].cpu().numpy(),
+                                        cnt[i, h].cpu().numpy(), tree.n_sel_levels)
+                err = H.max_abs(H.to64(O[0, i, h * G:(h + 1) * G]), cur.out)
+                assert err <= H.TOL_OUT["bf16"], f"row {t} head {h}: output max-abs {err}"
+    for h in range(Hkv):
+        H.compare_tree(tree, levels[h], 0, h, "bf16")
+
 def test_prefill_tensor_core_top_level(R):
     """Prefill on a tree with max_queries >= 128 scores the first scored level with
     one tensor-core product per group of rows.  The product's logits equal
