@@ -1180,11 +1180,20 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
     float* ll = mm + G * ns;     // [G][ns] l
     float* vals = ll + G * ns;   // [ns][E] staged values
     auto slot_of = [&](int i) { return i < nls ? i : NL * SPL + (i - nls); };
-    for (int x = threadIdx.x; x < ns * G; x += kThreads) {
-        const int i = x / G, g = x % G;
-        const float* rec = P + (slot_of(i) * G + g) * (D + 2);
-        mm[g * ns + i] = __ldcg(rec + D);
-        ll[g * ns + i] = __ldcg(rec + D + 1);
+    const int cap = (nbuf - 3 * G * ns) / ns;   // output elements staged per round
+    // (m, l) of every slot and head, and the first round of values, in one batch
+    const int E0 = min(cap, e1 - e0);
+    for (int x = threadIdx.x; x < ns * G + ns * E0; x += kThreads) {
+        if (x < ns * G) {
+            const int i = x / G, g = x % G;
+            const float* rec = P + (slot_of(i) * G + g) * (D + 2);
+            mm[g * ns + i] = __ldcg(rec + D);
+            ll[g * ns + i] = __ldcg(rec + D + 1);
+        } else {
+            const int y = x - ns * G;
+            const int i = y / E0, e = e0 + y % E0;
+            vals[y] = __ldcg(P + (slot_of(i) * G + e / D) * (D + 2) + e % D);
+        }
     }
     __syncthreads();
     for (int g = warp; g < G; g += kWarps) {
@@ -1203,14 +1212,14 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
         for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
         if (lane == 0) Lsh[g] = L;
     }
-    const int cap = (nbuf - 3 * G * ns) / ns;   // output elements staged per round
     for (int c0 = e0; c0 < e1; c0 += cap) {
         const int E = min(cap, e1 - c0);
         __syncthreads();   // the previous round's reads (and the weights) are done
-        for (int x = threadIdx.x; x < ns * E; x += kThreads) {
-            const int i = x / E, e = c0 + x % E;
-            vals[x] = __ldcg(P + (slot_of(i) * G + e / D) * (D + 2) + e % D);
-        }
+        if (c0 > e0)
+            for (int x = threadIdx.x; x < ns * E; x += kThreads) {
+                const int i = x / E, e = c0 + x % E;
+                vals[x] = __ldcg(P + (slot_of(i) * G + e / D) * (D + 2) + e % D);
+            }
         __syncthreads();
         for (int x = threadIdx.x; x < E; x += kThreads) {
             const int e = c0 + x, g = e / D;
