@@ -68,6 +68,42 @@ struct Dims<__nv_bfloat16, 2> {
     }
 };
 
+// One lane's DPL elements of a row as loaded (packed), widened when used, so a
+// batch of rows in flight costs one register per two bf16 elements.
+template <typename T, int N>
+struct Packed;
+template <>
+struct Packed<__nv_bfloat16, 4> {
+    uint2 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = *reinterpret_cast<const uint2*>(p); }
+    __device__ __forceinline__ float get(int e) const {
+        const uint32_t w = (e < 2) ? v.x : v.y;
+        return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+    }
+};
+template <>
+struct Packed<__nv_bfloat16, 2> {
+    uint32_t v;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = *reinterpret_cast<const uint32_t*>(p); }
+    __device__ __forceinline__ float get(int e) const {
+        return __uint_as_float((e & 1) ? (v & 0xffff0000u) : (v << 16));
+    }
+};
+template <>
+struct Packed<float, 4> {
+    float4 v;
+    __device__ __forceinline__ void load(const float* p) { v = *reinterpret_cast<const float4*>(p); }
+    __device__ __forceinline__ float get(int e) const {
+        return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+    }
+};
+template <>
+struct Packed<float, 2> {
+    float2 v;
+    __device__ __forceinline__ void load(const float* p) { v = *reinterpret_cast<const float2*>(p); }
+    __device__ __forceinline__ float get(int e) const { return e == 0 ? v.x : v.y; }
+};
+
 // softmax(w[0..m-1]) for every m = 1..C, fp64, into alpha[(m-1)*C + c].
 __device__ inline void fill_alpha(const float* w, int C, double* alpha) {
     for (int idx = threadIdx.x; idx < C * C; idx += blockDim.x) {
@@ -94,12 +130,12 @@ __device__ __forceinline__ void pool_rows(const T* sk, const T* sv, int64_t rs, 
     constexpr int N = PoolShape<T, D>::DPL;
     const int off = (threadIdx.x & 31) * N;
     for (int r0 = r_lo; r0 < r_hi; r0 += B) {
-        float kx[B][N], vx[B][N];
+        Packed<T, N> kx[B], vx[B];
 #pragma unroll
         for (int u = 0; u < B; ++u)
             if (r0 + u < r_hi) {
-                Dims<T, N>::load(sk + (r0 + u) * rs + off, kx[u]);
-                Dims<T, N>::load(sv + (r0 + u) * rs + off, vx[u]);
+                kx[u].load(sk + (r0 + u) * rs + off);
+                vx[u].load(sv + (r0 + u) * rs + off);
             }
 #pragma unroll
         for (int u = 0; u < B; ++u)
@@ -107,8 +143,8 @@ __device__ __forceinline__ void pool_rows(const T* sk, const T* sv, int64_t rs, 
                 const double al = alpha_m[r0 + u];
 #pragma unroll
                 for (int e = 0; e < N; ++e) {
-                    ak[e] = fma(al, (double)kx[u][e], ak[e]);
-                    av[e] += (double)vx[u][e];
+                    ak[e] = fma(al, (double)kx[u].get(e), ak[e]);
+                    av[e] += (double)vx[u].get(e);
                 }
             }
     }
@@ -140,7 +176,8 @@ __device__ __forceinline__ void warp_pool_node(const T* sk, const T* sv, int64_t
     double ak[N], av[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) { ak[e] = 0.0; av[e] = 0.0; }
-    pool_rows<T, D>(sk, sv, rs, 0, m, alpha_m, ak, av);
+    // every child row of a node in flight at once when rows pack two bf16 per word
+    pool_rows<T, D, sizeof(T) == 2 ? 16 : 8>(sk, sv, rs, 0, m, alpha_m, ak, av);
     float fk[N], fv[N];
     pool_store<T, D>(ak, av, m, dk, dv, fk, fv);
 }
