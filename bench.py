@@ -32,11 +32,11 @@ METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
 # capture at batch 1 (profiles/pass_kernel_decode524k_b1.md); a launch covers
 # batch x 8 independent units, so the batch-B figure is B times this.  Valid only
 # for the kernel sources it was taken from: any edit to them turns it into null.
-TRAFFIC_PASS_B1 = {"bytes": 44_200_192 + 97_280,
+TRAFFIC_PASS_B1 = {"bytes": 44_201_728 + 149_504,
                    "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
                                "long_context_recsa_b200/csrc/recsa_internal.cuh",
                                "long_context_recsa_b200/csrc/pool.cuh"],
-                   "sha256": "6af08ff33e762e2c55e88191f42f57db361298b87ef1c50d765746fe8b7d4cdf"}
+                   "sha256": "c241b4a737f4525f8e07d150c3d882357917f2c18e17851d3510d574f79065e4"}
 
 
 def captured_traffic(kernel: str, batch: int):
