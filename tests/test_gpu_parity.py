@@ -212,8 +212,9 @@ def test_host_errors_are_returned_not_launched(R):
 
 @pytest.mark.parametrize("k,L", [(128, 40000), (64, 30000)])
 def test_long_lists_sampled_select(R, k, L):
-    """Lists of 1024-2048 entries: the selection runs on a compact candidate list
-    bounded by a sampled threshold; sets must still be exact."""
+    """Lists of 1024-2048 entries spread over a cluster's CTAs: the distributed
+    histogram, the published boundary-bin candidates and the list-order ranks across
+    CTAs; sets must still be exact."""
     run_decode_case(R, config_id=17, B=2, Hkv=2, Hq=8, d=128, C=16, k=k, lengths=[L, L - 777],
                     dtype="bf16", cap=L, n_needles=16)
 
