@@ -178,6 +178,19 @@ RECSA_API recsa_status recsa_prefill_chunk(recsa_tree* tree, const void* Q, int6
  * the first device-side error recorded since the last call. */
 RECSA_API recsa_status recsa_get_status(recsa_tree* tree, void* stream);
 
+/* Self-test of the device-side timeout path.  Runs one CTA that waits, through the
+ * same bounded mbarrier wait every kernel of the library uses, on a barrier that
+ * nothing completes.  The wait gives up after its poll limit (about one second),
+ * records the timeout in `status_dev` and the kernel returns; no GPU fault, trap or
+ * hang is involved.
+ *   status_dev  device pointer to one uint32, caller-owned; zeroed here, then
+ *               written by the kernel (3 = timeout);
+ *   stream      the stream to run on, synchronised before returning.
+ * Returns RECSA_E_TIMEOUT when the wait gave up as designed, RECSA_OK if it did not
+ * (the path is broken), RECSA_E_INVAL for a NULL pointer, RECSA_E_CUDA on a CUDA
+ * error. */
+RECSA_API recsa_status recsa_probe_bounded_wait(uint32_t* status_dev, void* stream);
+
 typedef struct {
     int32_t n_levels;       /* levels stored at capacity, level 0 included           */
     int32_t n_sel_levels;   /* NL: highest level that any position can score         */

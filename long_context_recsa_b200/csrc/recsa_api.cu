@@ -215,6 +215,11 @@ static recsa_status finish_walk(recsa_tree* t, cudaStream_t stream) {
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 
+namespace recsa {
+// tree_kernels.cu: the bounded-wait self-test kernel
+cudaError_t launch_bounded_wait_probe(uint32_t* status, cudaStream_t s);
+}  // namespace recsa
+
 extern "C" {
 
 const char* recsa_status_str(recsa_status s) {
@@ -477,6 +482,18 @@ recsa_status recsa_get_status(recsa_tree* t, void* stream) {
         case kStatusTimeout: return RECSA_E_TIMEOUT;
         default: return RECSA_E_DEVICE;
     }
+}
+
+recsa_status recsa_probe_bounded_wait(uint32_t* status_dev, void* stream) {
+    if (!status_dev) return RECSA_E_INVAL;
+    const cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(status_dev, 0, sizeof(uint32_t), s) != cudaSuccess) return RECSA_E_CUDA;
+    if (launch_bounded_wait_probe(status_dev, s) != cudaSuccess) return RECSA_E_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, status_dev, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return RECSA_E_CUDA;
+    return v == kStatusTimeout ? RECSA_E_TIMEOUT : RECSA_OK;
 }
 
 recsa_status recsa_tree_info(const recsa_tree* t, recsa_tree_info_t* info) {

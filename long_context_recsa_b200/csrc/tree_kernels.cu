@@ -212,6 +212,21 @@ __global__ void __launch_bounds__(256) append_walk_kernel(TreeView tv, WorkView 
     ancestor_walk<T, D>(tv, b, h, t, pre, alpha);
 }
 
+// Waits on an mbarrier that nothing arrives on, through the bounded wait of every
+// kernel here: the wait gives up, records the timeout in *status and returns.
+__global__ void bounded_wait_probe_kernel(uint32_t* status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) mbar_init(&bar, 1);
+    mbar_fence_init();
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0u, status);
+}
+
+cudaError_t launch_bounded_wait_probe(uint32_t* status, cudaStream_t s) {
+    bounded_wait_probe_kernel<<<1, 32, 0, s>>>(status);
+    return cudaGetLastError();
+}
+
 // ----------------------------------------------------------------------------
 // host launchers
 // ----------------------------------------------------------------------------

@@ -73,6 +73,7 @@ def _load():
         "recsa_set_profile_events": [P, I32, P, P],
         "recsa_decode_noalloc": [ctypes.POINTER(RecsaConfigC), I64, I32, P, P, ctypes.POINTER(I64),
                                  P, SZ, ctypes.POINTER(I64), P, P, P],
+        "recsa_probe_bounded_wait": [P, P],
         "recsa_tree_free": [P],
         "recsa_status_str": [I32],
     }

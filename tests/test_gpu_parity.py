@@ -369,3 +369,16 @@ def test_single_appends_without_decode_equal_build(R, dtype):
     ref = tables_equal(n)
     assert torch.equal(out, ref.decode(q)[0])
     assert inc.recsa_get_status() == R.RECSA_OK
+
+
+def test_bounded_wait_gives_up_and_reports_timeout(R):
+    """The device-side timeout path: a wait on an mbarrier that nothing completes
+    gives up after its poll limit and records the timeout; the context stays usable
+    (a decode afterwards is still correct)."""
+    import ctypes
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = R.lib.recsa_probe_bounded_wait(ctypes.c_void_p(st.data_ptr()), None)
+    assert rc == R.RECSA_E_TIMEOUT
+    assert int(st.item()) == 3
+    run_decode_case(R, config_id=21, B=1, Hkv=1, Hq=2, d=64, C=4, k=3, lengths=[300],
+                    dtype="f32", cap=300)
