@@ -9,6 +9,7 @@ which are not available here):
   * K, V, q ~ N(0, 1), drawn in fp32 by ``torch.randn`` and rounded to the
     storage dtype (round to nearest even).
   * pooler logits w in R^C ~ N(0, 1) from the CPU generator, seed 7.
+  * gated-pooler parameters (Eq.5, forward only): seeded stand-ins, seed 11.
   * needles: seeded positions whose keys are set to ``gain`` times the mean of
     the GQA group's query heads (before RoPE), so that selection is non-trivial.
   * seed of a slice = 1_000_000*config + 10_000*stream + 100*sequence + head;
@@ -44,6 +45,26 @@ def pooler_w(C: int, seed: int = 7) -> torch.Tensor:
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     return torch.randn(C, generator=g, dtype=torch.float32)
+
+
+def gated_pooler_params(d: int, hidden: int | None = None, seed: int = 11) -> dict:
+    """Seeded stand-in parameters of the gated pooler (trained values are not
+    available): w, tau, g, rho and the MLP W1 [hidden][2d], b1 [hidden], W2
+    [d][hidden], drawn on the CPU generator and returned as fp64 tensors/floats.
+    Scales keep the pooled keys of N(0, 1) children O(1)."""
+    h = d if hidden is None else hidden
+    gen = torch.Generator().manual_seed(seed)
+    def nrm(*shape, std):
+        return (torch.randn(*shape, generator=gen, dtype=torch.float64) * std)
+    return {
+        "w": nrm(d, std=d ** -0.5),
+        "tau": 2.0,
+        "g": 0.75,
+        "rho": float(d) ** 0.5,
+        "W1": nrm(h, 2 * d, std=(2 * d) ** -0.5),
+        "b1": nrm(h, std=0.1),
+        "W2": nrm(d, h, std=0.1 * h ** -0.5),
+    }
 
 
 def kv_slice(config: int, seq: int, head: int, L: int, d: int, dtype: str, device="cpu"):

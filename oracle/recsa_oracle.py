@@ -29,6 +29,11 @@ Readings where the pages are silent (each also listed in the design notes):
   * ties in TopK go to the lower node index.
   * summaries enter Eq.4 with their per-head logits and no count bias.
 
+Eq.5 ("Pooler Distillation"): ``gated_pool_keys`` / ``build_tree_gated``, the
+gated key pooler, forward only, with seeded stand-in parameters (its readings are
+listed beside it).  It has no CUDA counterpart yet; its pins are in
+``tests/test_oracle_gated_pooler.py``.
+
 Parity pins: see ``tests/test_oracle_pins.py`` (closed forms for summary values
 and pooled keys, the C*k distance bound, the partition of [0..t] by the
 attended entries, dense-attention reduction when k exceeds every list, the
@@ -127,6 +132,79 @@ def build_tree(K0, V0, C: int, w, dtype: str):
     levels = [(K, V)]
     while levels[-1][0].shape[0] > 1:
         levels.append(pool_level(levels[-1][0], levels[-1][1], C, w, dtype))
+    return levels
+
+
+# ---------------------------------------------------------------------------
+# Eq.5 gated pooler ("Pooler Distillation"), forward only
+# ---------------------------------------------------------------------------
+# Readings where the pages leave the step open (also in the design notes):
+#   * x_c are the node's present children's stored keys (m <= C of them);
+#   * mu = their mean (a vector); sigma = their scalar spread about mu, the root
+#     of the mean squared deviation over children and dimensions, plus GATED_EPS
+#     inside the root so that identical children give a finite result;
+#   * g, tau, rho are scalars; w in R^d; the MLP has hidden width h (a parameter),
+#     W1 [h][2d], b1 [h], W2 [d][h] and no output bias;
+#   * values keep Eq.1: the mean of the children's values;
+#   * the result is rounded once to the storage dtype, as for Eq.1.
+GATED_EPS = 1e-6
+
+
+def _silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def gated_pool_keys(X: np.ndarray, P: dict) -> np.ndarray:
+    """Eq.5 for nodes given as X [n][m][d] (n nodes of m present children each):
+    alpha = softmax_c(tau w.(x_c - mu) / sigma), p = sum_c alpha_c x_c,
+    m = W2 SiLU(W1 [mu/rho ; (p - mu)/sigma] + b1), K = mu + g (p - mu) + sigma m.
+    Returns [n][d] in fp64 (not rounded)."""
+    X = np.asarray(X, dtype=np.float64)
+    n, mc, d = X.shape
+    w = np.asarray(P["w"], dtype=np.float64)
+    W1 = np.asarray(P["W1"], dtype=np.float64)
+    b1 = np.asarray(P["b1"], dtype=np.float64)
+    W2 = np.asarray(P["W2"], dtype=np.float64)
+    tau, g, rho = float(P["tau"]), float(P["g"]), float(P["rho"])
+    mu = X.mean(axis=1)                                               # [n][d]
+    dev = X - mu[:, None, :]
+    sigma = np.sqrt((dev ** 2).sum(axis=(1, 2)) / (mc * d) + GATED_EPS)   # [n]
+    logits = tau * (dev @ w) / sigma[:, None]                         # [n][m]
+    logits -= logits.max(axis=1, keepdims=True)
+    a = np.exp(logits)
+    a /= a.sum(axis=1, keepdims=True)
+    p = np.einsum("nc,ncd->nd", a, X)
+    z = np.concatenate([mu / rho, (p - mu) / sigma[:, None]], axis=1)    # [n][2d]
+    mlp = _silu(z @ W1.T + b1) @ W2.T                                  # [n][d]
+    return mu + g * (p - mu) + sigma[:, None] * mlp
+
+
+def pool_level_gated(Kc: np.ndarray, Vc: np.ndarray, C: int, P: dict, dtype: str):
+    """One level of the tree with the Eq.5 key pooler: parent i has children
+    C*i .. min(C*i+C-1, n-1); K_i by Eq.5 over them, V_i their mean; both rounded
+    to the storage dtype."""
+    n, d = Kc.shape
+    n_par = -(-n // C)
+    Kp = np.empty((n_par, d))
+    Vp = np.empty((n_par, d))
+    full = n // C
+    if full:
+        Kp[:full] = gated_pool_keys(Kc[: full * C].reshape(full, C, d), P)
+        Vp[:full] = Vc[: full * C].reshape(full, C, d).sum(axis=1) / C
+    if n_par > full:                       # ragged last node
+        m = n - full * C
+        Kp[full] = gated_pool_keys(Kc[full * C:][None], P)[0]
+        Vp[full] = Vc[full * C:].sum(axis=0) / m
+    return storage_round(Kp, dtype), storage_round(Vp, dtype)
+
+
+def build_tree_gated(K0, V0, C: int, P: dict, dtype: str):
+    """build_tree with the Eq.5 key pooler at every level."""
+    K = storage_round(K0, dtype)
+    V = storage_round(V0, dtype)
+    levels = [(K, V)]
+    while levels[-1][0].shape[0] > 1:
+        levels.append(pool_level_gated(levels[-1][0], levels[-1][1], C, P, dtype))
     return levels
 
 
