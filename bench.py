@@ -43,7 +43,7 @@ def captured_traffic(kernel: str, batch: int):
     """Per-launch DRAM traffic of `kernel` at this batch, or None when no capture of
     the current sources exists."""
     import hashlib
-    if kernel != "pass_kernel" or TRAFFIC_PASS_B1["bytes"] is None:
+    if kernel != "pass_kernel" or TRAFFIC_PASS_B1["bytes"] is None or W["L"] != 524288:
         return None
     h = hashlib.sha256()
     here = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +71,9 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--batch", type=int, default=4,
                    help="sequences per GPU (the headline workload uses 4)")
+    p.add_argument("--context", type=int, default=524288,
+                   help="context length (the headline workload uses 524288; 131072 and "
+                        "2097152 are the other decode configurations, reported only)")
     return p.parse_args(argv)
 
 
@@ -200,7 +203,8 @@ def max_over_ranks(x, ws, device: str = "cuda"):
 
 def workload_config(B: int, ws: int) -> dict:
     """The bench's workload, named by what it is (both arms report this)."""
-    return {"workload": f"decode 524K ctx, batch {B}, append 1 token/seq/step, "
+    ctx = {131072: "131K", 524288: "524K", 2097152: "2M"}.get(W["L"], str(W["L"]))
+    return {"workload": f"decode {ctx} ctx, batch {B}, append 1 token/seq/step, "
                         "Hq=32 Hkv=8 d=128 C=16 k=256 bf16",
             "seq_len": W["L"], "global_batch": B * ws, "parallelism": f"replicas x{ws}",
             "l2": "flushed (256 MB write) before every timed step",
@@ -229,6 +233,7 @@ def barrier(ws):
 def run_ours(args):
     import torch
     W["B"] = args.batch
+    W["L"] = args.context
     from long_context_recsa_b200 import build, inputs as I
     build.build()
     import long_context_recsa_b200.recsa as R
@@ -356,7 +361,8 @@ def run_ours(args):
                      "avg_launch_ms": round(kern_avg[dom], 5)},
         "kernel_ms": {("append" if w == -1 else "pass"):
                       (round(v, 5) if v else None) for w, v in kern_avg.items()},
-        "build_524k": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1)},
+        "build": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1),
+                  "tokens_per_seq": W["L"], "sequences": B},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
@@ -516,6 +522,7 @@ def run_reference(args):
     if rank != 0:
         return   # the oracle runs on rank 0 only; the other ranks exit without work
     W["B"] = args.batch
+    W["L"] = args.context
     import numpy as np
     from long_context_recsa_b200 import inputs as I
     from oracle import recsa_oracle as O
