@@ -37,7 +37,9 @@ listed beside it).  It has no CUDA counterpart yet; its pins are in
 Parity pins: see ``tests/test_oracle_pins.py`` (closed forms for summary values
 and pooled keys, the C*k distance bound, the partition of [0..t] by the
 attended entries, dense-attention reduction when k exceeds every list, the
-q = 0 tie-break, needles).  No function here is "parity unpinned".
+q = 0 tie-break, needles, the GQA group-mean importance against a brute-force
+selection with disagreeing heads, and per-head token weights of Eq.4 with
+several heads).  No function here is "parity unpinned".
 """
 from __future__ import annotations
 

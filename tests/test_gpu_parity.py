@@ -24,13 +24,15 @@ def R():
 
 
 def run_decode_case(R, *, config_id, B, Hkv, Hq, d, C, k, lengths, dtype, cap=None,
-                    n_needles=0, base=1e6, check_units=None, check_tree=True):
+                    n_needles=0, base=1e6, check_units=None, check_tree=True, q_fn=None):
     cap = cap or max(lengths)
     w = H.w_for(C)
     cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype=dtype,
                    rope_base=base, pooler_w=w)
     K, V, q = H.make_inputs(config_id, B, Hkv, Hq, d, cap, lengths, dtype, n_needles=n_needles)
     q = q[:, 0].contiguous()
+    if q_fn is not None:
+        q = q_fn(q).contiguous()
     tree = R.RecsaTree(cfg, cap, B, k0=K, v0=V)
     tree.recsa_build(lengths)
     out, sel, cnt = tree.decode(q, with_sel=True)
@@ -73,6 +75,28 @@ def test_small_ragged_batches(R, dtype, C, k, d, G):
     lengths = [1000, 777, 64 * C + 1, 5]
     run_decode_case(R, config_id=11, B=4, Hkv=Hkv, Hq=G * Hkv, d=d, C=C, k=k, lengths=lengths,
                     dtype=dtype, cap=1100, n_needles=3)
+
+
+def test_gqa_heads_that_disagree(R):
+    """G = 4 query heads per KV head whose logits disagree (head 1 ~ -head 0, heads 2
+    and 3 other directions): the selection follows the mean of the group's logits,
+    which no single head's ranking gives, and each head keeps its own logits in the
+    unified softmax."""
+    G = 4
+
+    def disagree(q):
+        g = torch.Generator(device="cpu").manual_seed(4242)
+        noise = torch.randn(q.shape, generator=g).to(q.device, q.dtype)
+        qg = q.view(q.shape[0], -1, G, q.shape[-1]).clone()
+        nz = noise.view_as(qg)
+        qg[:, :, 1] = -qg[:, :, 0] + 0.4 * nz[:, :, 1]
+        qg[:, :, 3] = -qg[:, :, 2] + 0.4 * nz[:, :, 3]
+        return qg.view_as(q)
+
+    run_decode_case(R, config_id=22, B=2, Hkv=2, Hq=2 * G, d=128, C=16, k=16,
+                    lengths=[5000, 4321], dtype="bf16", cap=5000, q_fn=disagree)
+    run_decode_case(R, config_id=22, B=1, Hkv=1, Hq=G, d=64, C=16, k=16, lengths=[5000],
+                    dtype="f32", cap=5000, q_fn=disagree)
 
 
 @pytest.mark.parametrize("L", [1, 2, 15, 16, 17, 255, 256, 257, 4095, 4096, 4097, 6000])

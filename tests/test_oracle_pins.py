@@ -367,3 +367,105 @@ def test_forced_selection_reproduces_own_choice():
     forced = {tr.level: tr.S for tr in res.levels if tr.scored}
     res2 = O.select_and_attend(lv, q, n - 1, C, k, forced=forced)
     np.testing.assert_array_equal(res.out, res2.out)
+
+
+# --------------------------------------------------------------- GQA pins
+
+def _brute_selection(levels, q, t, C, k, base):
+    """Eq.3 top-down written out with explicit loops, for a GQA group q [G, d]:
+    per-head logits through the complex-number RoPE route at candidate-local
+    positions, importance = (1/G) * the sum over the group's heads, TopK by a
+    sort on (importance descending, node ascending), then the children of the kept
+    nodes.  Returns {level: S} for the scored levels and {0: A^(0)}."""
+    G, d = q.shape
+    top = len(levels) - 1
+    a = [t // C ** l for l in range(top + 1)]
+    A = list(range(a[top] + 1))
+    out = {}
+    for l in range(top, 0, -1):
+        if len(A) > k:
+            p_q = len(A) - 1
+            qr = [_rope_complex(q[g], p_q, base) for g in range(G)]
+            imp = {}
+            for pos, node in enumerate(A[:-1]):
+                kr = _rope_complex(levels[l][0][node], pos, base)
+                tot = 0.0
+                for g in range(G):
+                    tot += float(np.dot(qr[g], kr)) / math.sqrt(d)
+                imp[node] = tot / G
+            ranked = sorted(A[:-1], key=lambda n: (-imp[n], n))
+            S = sorted(ranked[: k - 1]) + [A[-1]]
+            out[l] = S
+        else:
+            S = A
+        A = [c for i in S for c in range(C * i, min(C * i + C - 1, a[l - 1]) + 1)]
+    out[0] = A
+    return out
+
+
+def test_gqa_importance_is_the_group_mean_against_brute_force():
+    """The importance of Eq.3 for a GQA group is the mean of its heads' logits
+    (the stand-in for the importance the pages do not define).  Two heads that
+    disagree (q1 ~ -q0) make the mean's ranking differ from either head's own, so
+    selecting by one head, or by anything but the mean, changes some S; the oracle's
+    sets must equal the brute-force mean selection at every scored level."""
+    C, k, n, d = 4, 5, 1500, 16
+    r = np.random.default_rng(31)
+    K = r.standard_normal((n, d))
+    V = r.standard_normal((n, d))
+    lv = O.build_tree(K, V, C, r.standard_normal(C), "f64")
+    q0 = r.standard_normal(d)
+    q = np.stack([q0, -q0 + 0.4 * r.standard_normal(d)])
+    base = 1e4
+    differs_from_single_head = set()
+    for t in (n - 1, 1234, 777):
+        res = O.select_and_attend(lv, q, t, C, k, base=base)
+        want = _brute_selection(lv, q, t, C, k, base)
+        by_head = [_brute_selection(lv, q[[g]], t, C, k, base) for g in range(2)]
+        scored = [tr for tr in res.levels if tr.scored]
+        assert scored and sorted(want) == sorted([tr.level for tr in scored] + [0])
+        for tr in scored:
+            np.testing.assert_array_equal(tr.S, want[tr.level], err_msg=f"t={t} level {tr.level}")
+            for g in range(2):
+                if list(by_head[g][tr.level]) != list(want[tr.level]):
+                    differs_from_single_head.add(g)
+        np.testing.assert_array_equal(res.A0, want[0])
+    # the case has teeth: each head alone would have chosen differently somewhere
+    assert differs_from_single_head == {0, 1}
+
+
+def test_token_weights_per_head_with_gqa():
+    """Eq.4 indexes the logits by head: with G = 3 heads sharing one selection and
+    V = identity rows, row h of the output is the weight head h's own softmax gives
+    every token (a summary's weight split equally over its tokens), recomputed here
+    from that head's logits via the complex-number RoPE route."""
+    C, k, d, n, G = 2, 2, 64, 64, 3
+    r = np.random.default_rng(17)
+    K = r.standard_normal((n, d))
+    V = np.eye(n, d)
+    lv = O.build_tree(K, V, C, r.standard_normal(C), "f64")
+    q = r.standard_normal((G, d)) * np.array([[1.0], [2.0], [-1.5]])
+    t, base = n - 1, 1e4
+    res = O.select_and_attend(lv, q, t, C, k, base=base)
+    entries = []                       # (level, node, candidate-local position, p_q)
+    for tr in res.levels:
+        if tr.scored:
+            for pos, node in enumerate(tr.A[:-1]):
+                if node not in tr.S:
+                    entries.append((tr.level, node, pos, tr.p_q))
+    for pos, tok in enumerate(res.A0):
+        entries.append((0, tok, pos, len(res.A0) - 1))
+    assert any(e[0] > 0 for e in entries)
+    for h in range(G):
+        lg = np.array([_rope_complex(q[h], pq, base) @ _rope_complex(lv[l][0][node], pos, base)
+                       / math.sqrt(d) for l, node, pos, pq in entries])
+        p = np.exp(lg - lg.max())
+        p /= p.sum()
+        expect = np.zeros(n)
+        for pi, (l, node, _, _) in zip(p, entries):
+            span = np.arange(node * C ** l, (node + 1) * C ** l)
+            expect[span] += pi / len(span)
+        np.testing.assert_allclose(res.out[h], expect, rtol=1e-12, atol=1e-14,
+                                   err_msg=f"head {h}")
+    # heads with different queries get different weights (the pin can tell them apart)
+    assert np.abs(res.out[0] - res.out[1]).max() > 1e-3
