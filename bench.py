@@ -29,7 +29,7 @@ sys.path.insert(0, ROOT)
 METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
 
 # DRAM bytes (read + write) per launch of the select/attend pass kernel from one ncu
-# capture at batch 1 (profiles/pass_kernel_decode524k_b1.md); a launch covers
+# capture at batch 1 (the pass kernel's summary under profiles/); a launch covers
 # batch x 8 independent units, so the batch-B figure is B times this.  Valid only
 # for the kernel sources it was taken from: any edit to them turns it into null.
 TRAFFIC_PASS_B1 = {"bytes": 44_201_728 + 149_504,

@@ -174,8 +174,10 @@ RECSA_API recsa_status recsa_decode(recsa_tree* tree, const void* q, void* out, 
 RECSA_API recsa_status recsa_prefill_chunk(recsa_tree* tree, const void* Q, int64_t pos0, int32_t n,
                                  void* O, int32_t* sel_out, int32_t* counts_out, void* stream);
 
-/* Synchronise `stream`, read and clear the device status word.  Returns RECSA_OK or
- * the first device-side error recorded since the last call. */
+/* Run any pending ancestor re-pooling on `stream`, then read and clear the device
+ * status word in stream order (a copy and, if it was set, a clear on `stream`) and
+ * synchronise `stream` (not the device).  Returns RECSA_OK or the first device-side
+ * error recorded since the last call. */
 RECSA_API recsa_status recsa_get_status(recsa_tree* tree, void* stream);
 
 /* Self-test of the device-side timeout path.  Runs one CTA that waits, through the
@@ -246,6 +248,12 @@ RECSA_API recsa_status recsa_set_profile_events(recsa_tree* tree, int32_t which,
  *                          for these lengths, laid out as recsa_query_sizes states.
  *   lengths                host array [batch]; query b sits at lengths[b] - 1.
  *   q, out                 [batch][Hq][d] device, 16-byte aligned.
+ *   status_out             optional device uint32 (4-byte aligned), caller-owned: set
+ *                          to 0 at the start of the call, then to the first
+ *                          device-side error of this call (3: a bounded wait gave up,
+ *                          4: a staging buffer was misaligned).  Read it after the
+ *                          stream has reached the end of the call.  NULL: such errors
+ *                          are not reported.
  * Scratch: a fixed 8 MiB device array inside the library (held by every GPU that
  * loads it until exit), shared by all calls: calls that may overlap on the GPU race.
  * A shape whose workspace (recsa_query_sizes with max_queries = batch) exceeds 8 MiB
@@ -257,7 +265,8 @@ RECSA_API recsa_status recsa_decode_noalloc(const recsa_config* cfg, int64_t cap
                                             int32_t batch, const void* k0, const void* v0,
                                             const int64_t kv_strides[3], const void* levels,
                                             size_t level_bytes, const int64_t* lengths,
-                                            const void* q, void* out, void* stream);
+                                            const void* q, void* out, uint32_t* status_out,
+                                            void* stream);
 
 /* Free the host handle.  Device memory stays with the caller. */
 RECSA_API recsa_status recsa_tree_free(recsa_tree* tree);

@@ -16,6 +16,11 @@
 // race with each other.  Each call re-initialises everything it reads before reading
 // it (status word, lengths, RoPE table; selections and partials are fully written
 // before use), so a call never depends on what the previous call left behind.
+//
+// Device-side conditions (a bounded wait that gave up, a misaligned staging buffer)
+// are recorded in a status word: the caller's `status_out` when given (zeroed at the
+// start of the call, then written by the kernels), else a word inside the scratch
+// that nobody reads.
 #include <mutex>
 
 #include "recsa_internal.cuh"
@@ -53,9 +58,10 @@ using namespace recsa;
 extern "C" RECSA_API recsa_status recsa_decode_noalloc(
     const recsa_config* cfg, int64_t capacity, int32_t batch, const void* k0, const void* v0,
     const int64_t kv_strides[3], const void* levels, size_t level_bytes, const int64_t* lengths,
-    const void* q, void* out, void* stream) {
+    const void* q, void* out, uint32_t* status_out, void* stream) {
     if (!cfg || !lengths || !q || !out) return RECSA_E_INVAL;
-    if ((((uintptr_t)q) & 15u) || (((uintptr_t)out) & 15u)) return RECSA_E_INVAL;
+    if ((((uintptr_t)q) & 15u) || (((uintptr_t)out) & 15u) || (((uintptr_t)status_out) & 3u))
+        return RECSA_E_INVAL;
     size_t need = 0;
     TreeView tv;
     WorkView wv;
@@ -71,6 +77,7 @@ extern "C" RECSA_API recsa_status recsa_decode_noalloc(
     st = views_for(cfg, capacity, batch, batch, k0, v0, kv_strides, levels, level_bytes, scratch,
                    &need, &tv, &wv);
     if (st != RECSA_OK) return st;
+    if (status_out) wv.status = status_out;   // zeroed by the workspace set-up below
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = prepare_kernels(cfg->dtype, tv.D, tv.G, wv.SPL, wv.NS0, tv.C, tv.k);
     if (e == cudaSuccess) e = launch_init_workspace(tv, wv, cfg->rope_base, s);

@@ -469,13 +469,15 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
 
 recsa_status recsa_get_status(recsa_tree* t, void* stream) {
     if (!t) return RECSA_E_INVAL;
-    if (finish_walk(t, (cudaStream_t)stream) != RECSA_OK) return RECSA_E_CUDA;
-    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RECSA_E_CUDA;
+    const cudaStream_t s = (cudaStream_t)stream;
+    if (finish_walk(t, s) != RECSA_OK) return RECSA_E_CUDA;
     uint32_t v = 0;
-    if (cudaMemcpy(&v, t->wv.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    if (cudaMemcpyAsync(&v, t->wv.status, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
         return RECSA_E_CUDA;
-    if (v != 0 && cudaMemset(t->wv.status, 0, sizeof(v)) != cudaSuccess) return RECSA_E_CUDA;
-    if (cudaDeviceSynchronize() != cudaSuccess) return RECSA_E_CUDA;
+    if (v != 0 && (cudaMemsetAsync(t->wv.status, 0, sizeof(v), s) != cudaSuccess ||
+                   cudaStreamSynchronize(s) != cudaSuccess))
+        return RECSA_E_CUDA;
     switch (v) {
         case kStatusOk: return RECSA_OK;
         case kStatusCapacity: return RECSA_E_CAPACITY;

@@ -324,13 +324,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
     return ok != 0;
 }
-// Bounded wait for a phase of an mbarrier: gives up after kWaitPolls suspended
-// waits of up to kWaitHintNs each (about one second in total), records
-// kStatusTimeout and returns false.  Never waits forever.
+// Bounded wait for a phase of an mbarrier: gives up after `polls` suspended waits
+// of up to kWaitHintNs each (kWaitPolls: about one second in total), records
+// kStatusTimeout and returns false.  Never waits forever.  After one wait of a CTA
+// has given up, its later waits use kWaitPollsAfterFail (about 2 ms): long enough
+// for copies that are merely late to land before the CTA exits, short enough that
+// a unit whose copies never complete returns soon.
 constexpr uint32_t kWaitHintNs = 20000;
 constexpr uint32_t kWaitPolls = 50000;
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* status) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i)
+constexpr uint32_t kWaitPollsAfterFail = 100;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                                  uint32_t polls = kWaitPolls) {
+    for (uint32_t i = 0; i < polls; ++i)
         if (mbar_try_wait(bar, parity, kWaitHintNs)) return true;
     atomicCAS(status, 0u, 3u);
     return false;

@@ -150,7 +150,8 @@ enum { kMiscDigit = 0, kMiscAbove = 1, kMiscCount = 2, kMiscScan = 4 /* kWarps+1
        kMiscFloat = 16 /* 2*G floats */, kMiscLast = 40, kMiscN = 41,
        // cluster selection: published counts, gathered counts (one per CTA), scalars
        kMiscPubC = 48, kMiscPubA = 49, kMiscSB = 50, kMiscSBAbove = 51, kMiscMemN = 52,
-       kMiscTk = 53, kMiscTj = 54, kMiscGC = 64 /* 16 */, kMiscGA = 80 /* 16 */ };
+       kMiscTk = 53, kMiscTj = 54, kMiscGC = 64 /* 16 */, kMiscGA = 80 /* 16 */,
+       kMiscFailed = 100 /* a bounded wait of this CTA gave up */ };
 
 // Split cluster barrier: arrive (release) and, later, wait (acquire); every thread
 // of every CTA of the cluster takes both, in this order.
@@ -725,6 +726,7 @@ struct WarpRing {
     uint64_t* bars;
     int nsw, slot_bytes;
     uint32_t* status;
+    volatile int* failed;   // CTA-wide: set once any wait of the CTA has given up
 };
 
 // Issue block q: rows [first, first + cnt) of a table with row stride rs.  One lane.
@@ -760,10 +762,14 @@ __device__ __forceinline__ void ring_issue_map(const WarpRing& R, int q, const C
             : "memory");
 }
 
-// Wait (bounded) for block q; all lanes of the warp.
+// Wait (bounded) for block q; all lanes of the warp.  Once a wait of the CTA has
+// given up (the status word holds the timeout), later waits are short: the unit's
+// output is then garbage anyway, and the CTA must reach its exit soon rather than
+// spend a full limit on every remaining block.
 __device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int q) {
     const int s = q % R.nsw;
-    mbar_wait_bounded(&R.bars[s], (uint32_t)((q / R.nsw) & 1), R.status);
+    const uint32_t polls = *R.failed ? kWaitPollsAfterFail : kWaitPolls;
+    if (!mbar_wait_bounded(&R.bars[s], (uint32_t)((q / R.nsw) & 1), R.status, polls)) *R.failed = 1;
     return R.slots + (size_t)s * R.slot_bytes;
 }
 
@@ -1268,8 +1274,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (ci >= tv.B * tv.Hkv) return;
         double* alpha = reinterpret_cast<double*>(smem);
         double* pre = alpha + RECSA_MAX_C * RECSA_MAX_C;
-        for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
         pdl_wait();
+        for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
         const int b = ci / tv.Hkv, h = ci % tv.Hkv;
         const int64_t t = wv.lens[b] - 1;
         __syncthreads();
@@ -1319,10 +1325,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     cg::cluster_group cluster = cg::this_cluster();
     const int csize = (int)cluster.num_blocks();
     const int crank = (int)cluster.block_rank();
-    // inputs no earlier kernel writes: the query heads and the child rotations
-    // (staged while the previous kernel may still be finishing)
     const T* qrow = reinterpret_cast<const T*>(qv.q) + ((int64_t)gq * tv.Hq + kvh * G) * D;
-    stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
+    if (threadIdx.x == 0) misc[kMiscFailed] = 0;
     if (threadIdx.x < kWarps * nsw) mbar_init(&bars[threadIdx.x], 1);
     mbar_fence_init();
     if constexpr (SW) {
@@ -1361,7 +1365,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
+    // Nothing before this wait reads global memory that an earlier kernel may have
+    // written (only L2 prefetch hints go out above): the kernel just before may be
+    // the caller's own, writing q.
     pdl_wait();
+    stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
     const int64_t len = wv.lens[b];
     const int64_t t = (qv.mode == 0) ? len - 1 : qv.pos0 + (gq - b * qv.n_per_b);
     const bool valid = t >= 0 && t < len;
@@ -1485,7 +1493,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const bool pre = !L0 && qv.pre != nullptr && level == qv.pre_level && identity;
         const int nk = pre ? 0 : nw;   // blocks [0, nk) are K, [nk, nk + nw) are V
         const WarpRing R{ring + (size_t)warp * nsw * slot_bytes, bars + warp * nsw, nsw,
-                         slot_bytes, wv.status};
+                         slot_bytes, wv.status, misc + kMiscFailed};
         auto group_first = [&](int jb) -> int64_t {
             return identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
         };

@@ -204,8 +204,8 @@ __global__ void __launch_bounds__(256) append_walk_kernel(TreeView tv, WorkView 
     double* alpha = walk_smem;
     double* pre = walk_smem + RECSA_MAX_C * RECSA_MAX_C;
     const int b = blockIdx.x / tv.Hkv, h = blockIdx.x % tv.Hkv;
-    for (int i = threadIdx.x; i < tv.C * tv.C; i += blockDim.x) alpha[i] = wv.alpha[i];
     pdl_wait();
+    for (int i = threadIdx.x; i < tv.C * tv.C; i += blockDim.x) alpha[i] = wv.alpha[i];
     const int64_t t = wv.lens[b] - 1;
     __syncthreads();
     if (t < 1) return;

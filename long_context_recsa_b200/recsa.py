@@ -72,7 +72,7 @@ def _load():
         "recsa_host_lengths": [P, ctypes.POINTER(I64)],
         "recsa_set_profile_events": [P, I32, P, P],
         "recsa_decode_noalloc": [ctypes.POINTER(RecsaConfigC), I64, I32, P, P, ctypes.POINTER(I64),
-                                 P, SZ, ctypes.POINTER(I64), P, P, P],
+                                 P, SZ, ctypes.POINTER(I64), P, P, P, P],
         "recsa_probe_bounded_wait": [P, P],
         "recsa_tree_free": [P],
         "recsa_status_str": [I32],
@@ -149,18 +149,20 @@ def recsa_query_sizes(cfg: Config, capacity: int, batch: int, max_queries: int):
 
 def recsa_decode_noalloc(cfg: Config, capacity: int, k0: torch.Tensor, v0: torch.Tensor,
                          levels: torch.Tensor, lengths, q: torch.Tensor, out: torch.Tensor,
-                         stream=None) -> int:
+                         status_out: torch.Tensor | None = None, stream=None) -> int:
     """Decode with the library's fixed device scratch instead of a caller workspace
     (for callers that cannot allocate device memory at the call site).  Returns the
-    status code; the buffers are the caller's (k0, v0 and levels as built for a tree
-    of this capacity and batch)."""
+    status code of the host-side checks; the buffers are the caller's (k0, v0 and
+    levels as built for a tree of this capacity and batch).  status_out: optional
+    one-element 32-bit device tensor that receives the call's device-side status
+    (0 when nothing went wrong)."""
     c = cfg.to_c()
     batch = q.shape[0]
     lens = (ctypes.c_int64 * batch)(*[int(x) for x in lengths])
     strides = (ctypes.c_int64 * 3)(*k0.stride()[:3])
     return lib.recsa_decode_noalloc(ctypes.byref(c), capacity, batch, _ptr(k0), _ptr(v0), strides,
                                     _ptr(levels), levels.numel(), lens, _ptr(q), _ptr(out),
-                                    _stream(stream))
+                                    _ptr(status_out), _stream(stream))
 
 
 class RecsaTree:

@@ -5,7 +5,10 @@ for per-call scratch).  Its scratch is a fixed array inside the library.
 
 Checked through the C ABI against recsa_decode on the same buffers, on two calls in
 a row with different queries, so that nothing left over from one call leaks into
-the next.  This file is collected last on purpose."""
+the next.  Both run the same kernels on the same inputs, so the outputs must be
+equal bit for bit (which is inside the tolerance of the other parity tests).  The
+device-side status each call writes into the caller's status word is checked too.
+This file is collected last on purpose."""
 import ctypes
 
 import pytest
@@ -35,15 +38,19 @@ def test_noalloc_decode_matches_decode_on_two_calls(R, dtype):
     K, V, Q = H.make_inputs(21, B, Hkv, Hq, d, cap, lengths, dtype, q_rows=2, n_needles=4)
     tree = R.RecsaTree(cfg, cap, B, k0=K, v0=V)
     tree.recsa_build(lengths)
+    status = torch.full((1,), 77, dtype=torch.int32, device="cuda")
     for call in range(2):
         q = Q[:, call].contiguous()
         ref = tree.decode(q)[0]
         out = torch.full_like(q, float("nan"))
-        st = R.recsa_decode_noalloc(cfg, cap, K, V, tree.levels, lengths, q, out)
+        status.fill_(77)
+        st = R.recsa_decode_noalloc(cfg, cap, K, V, tree.levels, lengths, q, out, status)
         torch.cuda.synchronize()
         assert st == R.RECSA_OK, R.lib.recsa_status_str(st)
+        assert int(status.item()) == 0, f"call {call}: device status {int(status.item())}"
         err = (out.double() - ref.double()).abs().max().item()
         assert err <= H.TOL_OUT[dtype], f"call {call}: max-abs {err}"
+        assert torch.equal(out, ref), f"call {call}: not bitwise equal (max-abs {err})"
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(R):
