@@ -14,8 +14,7 @@
 //      exact radix select of the top k-1 (ties to the lower list position, which
 //      is the lower node index because lists are ascending);
 //   3. writes its part of S^(l) (rank = number of selected entries before it;
-//      the current node is last), prefetches the children of its selected nodes
-//      (the next level's rows) into L2, and accumulates the split-softmax partial
+//      the current node is last) and accumulates the split-softmax partial
 //      (max, sum, weighted V) of its unselected entries: the summaries.
 // Entry j of the next list is node C*S[j/C] + j%C, so lists are never
 // materialised.  Level 0 scores A^(0) the same way with every entry included; the
@@ -669,16 +668,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// cnt consecutive rows starting at row `first` of a table with row stride rs.
-template <typename T, int D>
-__device__ __forceinline__ void prefetch_rows(const T* base, int64_t rs, int64_t first, int cnt) {
-    constexpr uint32_t kRow = D * sizeof(T);
-    if (rs == D) {
-        prefetch_l2(base + first * D, cnt * kRow);
-    } else {
-        for (int c = 0; c < cnt; ++c) prefetch_l2(base + (first + c) * rs, kRow);
-    }
-}
 
 // 16 loaded bytes as VEC/2 fp32 pairs (elements 2i, 2i+1).
 template <typename T>
@@ -1507,12 +1496,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ring_issue<T, D>(R, qbase + q, q < nk ? kbase : vbase, rs, group_first(jb),
                                  min(C, j1 - jb));
         };
-        if (identity && rs == D && threadIdx.x == 0 && j1 > j0) {
-            // the first scored level was not prefetched by a level above: its chunk
-            // (contiguous rows j0..j1) goes to L2 ahead of the ring
-            prefetch_l2(kbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
-            prefetch_l2(vbase + (int64_t)j0 * D, (uint32_t)(j1 - j0) * kRow);
-        }
         if (lane == 0)
             for (int q = 0; q < nsw && q < nk + nw; ++q) issue(q);
 
@@ -1587,35 +1570,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 __syncthreads();
                 select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, mark);
             }
-            const T* nk_;
-            const T* nv_;
-            int64_t nrs;
-            if (level == 1) {
-                nk_ = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
-                nv_ = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
-                nrs = tv.s_t;
-            } else {
-                nk_ = level_k<T>(tv, level - 1, b, kvh);
-                nv_ = level_v<T>(tv, level - 1, b, kvh);
-                nrs = D;
-            }
             if (crank == 0 && threadIdx.x == 0) {
                 const int64_t cur = apow(t, level, C, lgC);
                 sel_ws[K1] = (int)cur;
                 if (sel_usr) sel_usr[K1] = (int)cur;
                 cluster.map_shared_rank(par_next, K1 / ppc_next)[K1] = (int)cur;
-                const int nch = (int)(apow(t, level - 1, C, lgC) - (int64_t)C * cur + 1);
-                prefetch_rows<T, D>(nk_, nrs, (int64_t)C * cur, nch);
-                prefetch_rows<T, D>(nv_, nrs, (int64_t)C * cur, nch);
             }
             __syncthreads();
-            // the children of this chunk's selected nodes are the next level's rows: to
-            // L2, each thread for its own entries, so the requests go out in parallel
-            for (int i = threadIdx.x; i < n_sc; i += kThreads)
-                if (flag[i]) {
-                    prefetch_rows<T, D>(nk_, nrs, (int64_t)C * nodes[i], C);
-                    prefetch_rows<T, D>(nv_, nrs, (int64_t)C * nodes[i], C);
-                }
+            // No L2 prefetch of the kept nodes' children here: bulk prefetches queue in
+            // the same TMA unit as the rings' copies, and delayed this level's value
+            // blocks and the next level's first blocks by more than they saved.
         }
 
         // 3. softmax partial over the unselected (level) or all (level 0) entries
