@@ -69,6 +69,8 @@ def parse(argv=None):
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-contexts", action="store_true",
+                   help="skip the 131K and 2M decode configurations (reported under 'contexts')")
     p.add_argument("--batch", type=int, default=4,
                    help="sequences per GPU (the headline workload uses 4)")
     p.add_argument("--context", type=int, default=524288,
@@ -84,6 +86,18 @@ def peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def fp32_alu_peak():
+    """Dense fp32 FMA rate of the CUDA cores, derived from unit counts and the clock:
+    148 SMs x 128 fp32 lanes x 2 FLOP per FMA x the measured max SM clock (MHz)."""
+    mhz = 1965.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    except Exception:
+        pass
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12, f"148 SMs x 128 fp32 lanes x 2 FLOP x {mhz:.0f} MHz"
 
 
 def tf32_peak():
@@ -370,6 +384,13 @@ def run_ours(args):
         res["e2e"] = e2e_decode(tree, R, knew, vnew, qs, args, ws, flush)
     if not args.no_prefill:
         res["prefill"] = bench_prefill(R, I, cfg, K, V, tree, args, ws, dev, flush)
+    if not args.no_contexts and ws == 1:
+        del graphs, tree
+        torch.cuda.empty_cache()
+        res["contexts"] = {
+            "131K": bench_context(R, I, cfg, 131072, 1, 200, dev, flush, rank),
+            "2M": bench_context(R, I, cfg, 2097152, 1, 1000, dev, flush, rank),
+        }
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(K, V, qs, cfg, R)
     if ws > 1:
@@ -449,6 +470,7 @@ def bench_prefill(R, I, cfg, K, V, tree_decode, args, ws, dev, flush):
     res = {"value": round(ws * nq / (ms / 1e3), 1), "unit": "tok/s", "ms_per_chunk": round(ms, 3),
            "workload": "4096-query chunk at positions 520192..524287 of a 524288-token tree, "
                        "batch 1, same shapes"}
+    res["roofline"] = prefill_roofline(R, pt, Q, L - nq, O, dev)
     if pt.tc_queries > 0:
         # the top level's tensor-core product: time the chunk's last one with events
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -487,13 +509,146 @@ def bench_prefill(R, I, cfg, K, V, tree_decode, args, ws, dev, flush):
     return res
 
 
+def prefill_roofline(R, pt, Q, pos0, O, dev):
+    """Roofline of the dominant prefill kernel: the select/attend pass over one group
+    of rows (the chunk's last, timed with events).  Its work is plain fp32 arithmetic
+    on the CUDA cores (scoring with the rotation, and the weighted value sums), so the
+    bound is the fp32 FMA rate.  FLOPs per (row, KV head) from the list counts the
+    kernel returns: every key scored on the CUDA cores costs the rotation (6 FLOP per
+    rotary pair, d/2 pairs) and G dot products (2d FLOP each); every summary or level-0
+    token costs G weighted sums (2d FLOP each).  Keys of a level scored by the
+    tensor-core product are not counted here.  Logical bytes (the same counting rule as
+    decode, reads that mostly hit L2 because the rows share the tree) are reported
+    beside it."""
+    import numpy as np
+    import torch
+    Hkv, G, d, k, C = W["Hkv"], W["Hq"] // W["Hkv"], W["d"], W["k"], W["C"]
+    nq = Q.shape[1]
+    nl = pt.n_sel_levels
+    cnt = torch.zeros(nq, Hkv, nl + 1, dtype=torch.int32, device=dev)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(); b_.record()
+    pt.recsa_set_profile_events(0, a, b_)
+    pt.recsa_prefill_chunk(Q, pos0, O, None, cnt)
+    torch.cuda.synchronize()
+    pt.recsa_set_profile_events(0, None, None)
+    launch_ms = a.elapsed_time(b_)
+    rows = pt.tc_queries if pt.tc_queries > 0 else min(nq, pt.max_queries)
+    c = cnt[nq - rows:].cpu().numpy().astype("int64")       # the last launch's rows
+    t_last = pos0 + nq - 1
+    lt = 0
+    p = t_last
+    while p > 0:
+        p //= C
+        if p >= k:
+            lt += 1
+    flops = 0
+    nbytes = 0
+    s_vec = d * 2
+    for lvl in range(1, nl + 1):
+        cl = c[:, :, lvl]
+        scored = cl > 0
+        keys = (cl - 1) * scored
+        summ = (cl - np.minimum(k, cl)) * scored
+        if not (pt.tc_queries > 0 and lvl == lt):
+            flops += int(keys.sum()) * (6 * (d // 2) + 2 * G * d)
+            nbytes += int(keys.sum()) * s_vec
+        flops += int(summ.sum()) * 2 * G * d
+        nbytes += int(summ.sum()) * s_vec
+    tok = c[:, :, 0]
+    flops += int(tok.sum()) * 2 * G * d
+    nbytes += int(tok.sum()) * 2 * s_vec
+    peak, src = fp32_alu_peak()
+    hbm, kind = peaks()
+    achieved = flops / (launch_ms / 1e3) / 1e12
+    return {"bound": "alu", "kernel": "pass_kernel (per-row levels of one group of rows)",
+            "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": src,
+            "rows_per_launch": int(rows), "flop_per_launch": int(flops),
+            "avg_launch_ms": round(launch_ms, 4),
+            "logical_bytes_per_launch": int(nbytes),
+            "logical_GB_per_s": round(nbytes / (launch_ms / 1e3) / 1e9, 1),
+            "logical_frac_of_hbm": round(nbytes / (launch_ms / 1e3) / 1e9 / hbm, 4),
+            "note": "logical bytes are the lists' reads; most hit L2 (rows share the tree)"}
+
+
+def bench_context(R, I, cfg, L, B, steps, dev, flush, rank):
+    """Decode at another context length: the tree built from raw K, V (timed), then
+    `steps` append+decode steps replayed from one captured graph, each timed with
+    events after an L2 flush.  Reports the median and mean step time, tokens/s, the
+    pass kernel's algorithmic bytes and their fraction of the HBM peak."""
+    import torch
+    import statistics as st
+    Hq, Hkv, d = W["Hq"], W["Hkv"], W["d"]
+    dt = I.torch_dtype(W["dtype"])
+    cap = L + steps + 16
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank_seed(I.slice_seed(5 if L > 524288 else 2, I.STREAM_K, 0, 0), rank))
+    K = torch.empty(B, Hkv, cap, d, dtype=dt, device=dev)
+    V = torch.empty_like(K)
+    for h in range(Hkv):   # per head, to bound the fp32 staging tensor
+        K[:, h] = torch.randn(B, cap, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+        V[:, h] = torch.randn(B, cap, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    knew = torch.randn(steps, B, Hkv, 1, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    vnew = torch.randn(steps, B, Hkv, 1, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    qs = torch.randn(steps, B, Hq, d, generator=g, device=dev, dtype=torch.float32).to(dt)
+    tree = R.RecsaTree(cfg, cap, B, k0=K, v0=V)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    tree.recsa_build([L] * B)
+    e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    build_bytes = B * Hkv * L * d * 2 * 2 * (1 + 1 / 15.0)
+    kst = torch.empty(B, Hkv, 1, d, dtype=dt, device=dev)
+    vst = torch.empty_like(kst)
+    qst = torch.empty(B, Hq, d, dtype=dt, device=dev)
+    out = torch.empty_like(qst)
+    cnt = torch.zeros(B, Hkv, tree.n_sel_levels + 1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gr, stream=stream):
+            tree.recsa_append(kst, vst)
+            tree.recsa_decode(qst, out, None, cnt)
+    torch.cuda.synchronize()
+    times = []
+    for i in range(steps):
+        kst.copy_(knew[i]); vst.copy_(vnew[i]); qst.copy_(qs[i])
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        gr.replay()
+        s1.record()
+        s1.synchronize()
+        times.append(s0.elapsed_time(s1))
+    assert tree.recsa_get_status() == R.RECSA_OK
+    by, per_level = step_bytes(cnt.cpu().numpy(), W["k"], d * 2, B, Hkv, Hq, d, 2)
+    hbm, _ = peaks()
+    timed = times[3:] if len(times) > 6 else times
+    ms_med, ms_mean = st.median(timed), sum(timed) / len(timed)
+    res = {"context": L, "batch": B, "steps": steps, "ms_per_step_median": round(ms_med, 5),
+           "ms_per_step_mean": round(ms_mean, 5), "tok_per_s": round(B / (ms_mean / 1e3), 1),
+           "bytes_per_step": int(by),
+           "hbm_frac_of_measured": round(by / (ms_mean / 1e3) / 1e9 / hbm, 4),
+           "build": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1)},
+           "timing": "per-step CUDA events around one graph replay (append + decode), "
+                     "L2 flushed before every step; the first 3 steps not averaged"}
+    del gr, tree, K, V
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(K, V, qs, cfg, R):
     """The fp64 oracle on a bounded sample: select + attend of decode queries of one
     (sequence, KV head) unit over its pre-built fp64 tree (tree build excluded)."""
     import numpy as np
     import torch
+    from threadpoolctl import threadpool_limits
     from oracle import recsa_oracle as O
     cores = len(os.sched_getaffinity(0))
+    threadpool_limits(limits=cores)   # the oracle's BLAS calls use every host core
     L, C, k, G, d = W["L"], W["C"], W["k"], W["Hq"] // W["Hkv"], W["d"]
     Kh = K[0, 0, :L].double().cpu().numpy()
     Vh = V[0, 0, :L].double().cpu().numpy()
