@@ -280,6 +280,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     build_ms = e0.elapsed_time(e1)
     build_bytes = B * Hkv * L * d * esize * 2 * (1 + 1 / 15.0)
+    gated = bench_gated_build(R, I, cfg, K, V, cap, B, L, dev)
 
     # one decode step = append + decode, captured once; device-side lengths make
     # the graph replayable step after step
@@ -377,6 +378,7 @@ def run_ours(args):
                       (round(v, 5) if v else None) for w, v in kern_avg.items()},
         "build": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1),
                   "tokens_per_seq": W["L"], "sequences": B},
+        "build_gated": gated,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
@@ -570,6 +572,35 @@ def prefill_roofline(R, pt, Q, pos0, O, dev):
             "logical_GB_per_s": round(nbytes / (launch_ms / 1e3) / 1e9, 1),
             "logical_frac_of_hbm": round(nbytes / (launch_ms / 1e3) / 1e9 / hbm, 4),
             "note": "logical bytes are the lists' reads; most hit L2 (rows share the tree)"}
+
+
+def bench_gated_build(R, I, cfg, K, V, cap, B, L, dev, hidden=64):
+    """The same tree built with the Eq.5 gated key pooler (seeded parameters, MLP
+    width `hidden`), timed with events: fp64 per-node statistics and MLP, one warp
+    per node."""
+    import numpy as np
+    import torch
+    P = I.gated_pooler_params(W["d"], hidden=hidden)
+    pd = {"hidden": hidden, "tau": P["tau"], "g": P["g"], "rho": P["rho"],
+          "w": P["w"].to(dev), "W1t": P["W1"].t().contiguous().to(dev),
+          "b1": P["b1"].to(dev), "W2t": P["W2"].t().contiguous().to(dev)}
+    tg = R.RecsaTree(cfg, cap, B, k0=K, v0=V)
+    tg.recsa_tree_set_gated_pooler(pd)
+    tg.recsa_build([L] * B)   # warm-up (kernel load, attribute set-up)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    tg.recsa_build([L] * B)
+    e1.record()
+    torch.cuda.synchronize()
+    assert tg.recsa_get_status() == R.RECSA_OK
+    ms = e0.elapsed_time(e1)
+    nodes = sum(B * W["Hkv"] * (-(-L // W["C"] ** l)) for l in range(1, 8) if -(-L // W["C"] ** (l - 1)) > 1)
+    del tg
+    torch.cuda.empty_cache()
+    return {"ms": round(ms, 3), "hidden": hidden, "nodes": int(nodes),
+            "ns_per_node": round(ms * 1e6 / nodes, 2),
+            "note": "Eq.5 gated key pooler, fp64, seeded parameters; values as Eq.1"}
 
 
 def bench_context(R, I, cfg, L, B, steps, dev, flush, rank):

@@ -268,6 +268,31 @@ RECSA_API recsa_status recsa_decode_noalloc(const recsa_config* cfg, int64_t cap
                                             const void* q, void* out, uint32_t* status_out,
                                             void* stream);
 
+/* Eq.5 ("Pooler Distillation"), forward only: the gated key pooler, used in place of
+ * the stand-in pooler by every later recsa_build and recsa_append on the tree (call
+ * recsa_build after switching).  For a node with present children x_1..x_m:
+ *   mu = mean_c x_c;  sigma = sqrt(mean over children and dims of (x - mu)^2 + 1e-6);
+ *   alpha = softmax_c(tau * w . (x_c - mu) / sigma);  p = sum_c alpha_c x_c;
+ *   K = mu + g (p - mu) + sigma * W2 SiLU(W1 [mu / rho ; (p - mu) / sigma] + b1).
+ * The node's value stays Eq.1's mean of the children's values.  Computed in fp64 with
+ * one rounding to the storage dtype; build and append give bit-identical trees.
+ *   hidden  h, the MLP's hidden width, 1..64 (the fp64 weights are staged in shared
+ *           memory); larger widths return RECSA_E_UNSUPPORTED.
+ *   w       device fp64 [d];  W1t device fp64 [2d][h] (W1 transposed);  b1 device
+ *           fp64 [h];  W2t device fp64 [h][d] (W2 transposed).  Caller-owned, 8-byte
+ *           aligned, kept alive and unchanged while the tree uses them.
+ * p == NULL switches back to the stand-in pooler.  The pages do not give the trained
+ * parameters; the tests use seeded ones. */
+typedef struct {
+    int32_t hidden;
+    double tau, g, rho;
+    const double* w;
+    const double* W1t;
+    const double* b1;
+    const double* W2t;
+} recsa_gated_pooler;
+RECSA_API recsa_status recsa_tree_set_gated_pooler(recsa_tree* tree, const recsa_gated_pooler* p);
+
 /* Free the host handle.  Device memory stays with the caller. */
 RECSA_API recsa_status recsa_tree_free(recsa_tree* tree);
 

@@ -201,6 +201,9 @@ struct recsa_tree {
     // a single-token append left the ancestors of the new tokens to re-pool: the next
     // decode does it in its level-0 launch, any other call first
     bool walk_pending;
+    // Eq.5 gated key pooler in place of the stand-in (recsa_tree_set_gated_pooler)
+    bool gated;
+    GatedView gv;
 };
 
 // Runs a pending ancestor re-pooling on `stream` (before a call that needs the
@@ -345,7 +348,14 @@ recsa_status recsa_build(recsa_tree* t, const int64_t* lengths, void* stream) {
     for (int b = 0; b < t->B; ++b)
         if (lengths[b] < 0 || lengths[b] > t->cap) return RECSA_E_CAPACITY;
     t->walk_pending = false;   // the build pools every node anew
-    cudaError_t e = launch_build(t->tv, t->wv, lengths, t->cfg.dtype, (cudaStream_t)stream);
+    cudaError_t e;
+    if (t->gated) {
+        e = launch_set_lengths(t->wv, lengths, t->B, (cudaStream_t)stream);
+        if (e == cudaSuccess)
+            e = launch_gated_levels(t->tv, t->wv, t->gv, 0, t->cfg.dtype, (cudaStream_t)stream);
+    } else {
+        e = launch_build(t->tv, t->wv, lengths, t->cfg.dtype, (cudaStream_t)stream);
+    }
     if (e != cudaSuccess) return RECSA_E_CUDA;
     for (int b = 0; b < t->B; ++b) t->host_len[b] = lengths[b];
     return RECSA_OK;
@@ -360,7 +370,12 @@ recsa_status recsa_append(recsa_tree* t, const void* k_new, const void* v_new, i
     const cudaStream_t s = (cudaStream_t)stream;
     if (finish_walk(t, s) != RECSA_OK) return RECSA_E_CUDA;
     cudaError_t e;
-    if (n == 1) {
+    if (t->gated) {
+        // rows at the old lengths, every level's nodes over them, then the lengths
+        e = launch_append_rows(t->tv, t->wv, k_new, v_new, n, t->cfg.dtype, s);
+        if (e == cudaSuccess) e = launch_gated_levels(t->tv, t->wv, t->gv, n, t->cfg.dtype, s);
+        if (e == cudaSuccess) e = launch_commit_lengths(t->wv, t->B, n, t->cap, s);
+    } else if (n == 1) {
         e = launch_append_token(t->tv, t->wv, k_new, v_new, t->cfg.dtype, s, &t->prof);
         if (e == cudaSuccess) t->walk_pending = true;
     } else {
@@ -464,6 +479,32 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
                                                      t->has_maps ? t->maps : nullptr);
         if (e != cudaSuccess) return RECSA_E_CUDA;
     }
+    return RECSA_OK;
+}
+
+recsa_status recsa_tree_set_gated_pooler(recsa_tree* t, const recsa_gated_pooler* p) {
+    if (!t) return RECSA_E_INVAL;
+    if (p == nullptr) {
+        t->gated = false;
+        return RECSA_OK;
+    }
+    if (!p->w || !p->W1t || !p->b1 || !p->W2t) return RECSA_E_INVAL;
+    if ((((uintptr_t)p->w) | ((uintptr_t)p->W1t) | ((uintptr_t)p->b1) | ((uintptr_t)p->W2t)) & 7u)
+        return RECSA_E_INVAL;
+    if (p->hidden < 1) return RECSA_E_INVAL;
+    if (p->hidden > kGatedMaxHidden) return RECSA_E_UNSUPPORTED;
+    if (!isfinite(p->tau) || !isfinite(p->g) || !isfinite(p->rho) || p->rho == 0.0)
+        return RECSA_E_INVAL;
+    t->walk_pending = false;   // (a pending stand-in walk is dropped: rebuild after switching)
+    t->gv.h = p->hidden;
+    t->gv.tau = p->tau;
+    t->gv.g = p->g;
+    t->gv.rho = p->rho;
+    t->gv.w = p->w;
+    t->gv.W1t = p->W1t;
+    t->gv.b1 = p->b1;
+    t->gv.W2t = p->W2t;
+    t->gated = true;
     return RECSA_OK;
 }
 

@@ -39,6 +39,17 @@ struct TreeView {
     float w[RECSA_MAX_C];      // pooler logits; kernels form softmax(w[0..m-1]) in fp64
 };
 
+// Parameters of the Eq.5 gated key pooler (caller-owned fp64 device arrays).
+constexpr int kGatedMaxHidden = 64;
+struct GatedView {
+    int h;                     // MLP hidden width, 1..kGatedMaxHidden
+    double tau, g, rho;
+    const double* w;           // [D]
+    const double* W1t;         // [2D][h]  (W1 transposed)
+    const double* b1;          // [h]
+    const double* W2t;         // [h][D]   (W2 transposed)
+};
+
 // Which queries a select/attend launch handles.
 struct QueryView {
     const void* q;             // [Qtot][Hq][D]
@@ -371,6 +382,15 @@ inline bool uses_kv_maps(int dtype, int D, int C) {
 cudaError_t encode_kv_maps(const TreeView& tv, KVMaps* maps);
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype);
 cudaError_t launch_set_lengths(const WorkView& wv, const int64_t* lengths, int B, cudaStream_t s);
+// Eq.5 levels 1.. with the gated key pooler: every node (add == 0) or the nodes
+// covering the `add` tokens appended at the device-side lengths (gated.cu).
+cudaError_t launch_gated_levels(const TreeView& tv, const WorkView& wv, const GatedView& gv,
+                                int64_t add, int dtype, cudaStream_t s);
+// The single-token and multi-token append helpers of tree_kernels.cu.
+cudaError_t launch_append_rows(const TreeView& tv, const WorkView& wv, const void* k_new,
+                               const void* v_new, int n, int dtype, cudaStream_t s);
+cudaError_t launch_commit_lengths(const WorkView& wv, int B, int64_t add, int64_t cap,
+                                  cudaStream_t s);
 recsa_status views_for(const recsa_config* cfg, int64_t cap, int B, int Qmax, const void* k0,
                        const void* v0, const int64_t strides[3], const void* levels,
                        size_t level_bytes, char* ws, size_t* ws_bytes, TreeView* tv,

@@ -350,6 +350,28 @@ cudaError_t launch_append_walk(const TreeView& tv, const WorkView& wv, int dtype
     RECSA_DISPATCH_TD(dtype, tv.D, append_walk_impl, tv, wv, s);
 }
 
+template <typename T, int D>
+static cudaError_t append_rows_impl(const TreeView& tv, const WorkView& wv, const void* k_new,
+                                   const void* v_new, int n, cudaStream_t s) {
+    const int per_row = D / VecOf<T>::N;
+    int64_t blocks = ((int64_t)n * per_row + 255) / 256;
+    if (blocks > 1024) blocks = 1024;
+    append_rows_kernel<T, D><<<dim3((unsigned)blocks, tv.B * tv.Hkv), 256, 0, s>>>(
+        tv, wv, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new), n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append_rows(const TreeView& tv, const WorkView& wv, const void* k_new,
+                               const void* v_new, int n, int dtype, cudaStream_t s) {
+    RECSA_DISPATCH_TD(dtype, tv.D, append_rows_impl, tv, wv, k_new, v_new, n, s);
+}
+
+cudaError_t launch_commit_lengths(const WorkView& wv, int B, int64_t add, int64_t cap,
+                                  cudaStream_t s) {
+    commit_lengths_kernel<<<1, RECSA_MAX_BATCH, 0, s>>>(wv, B, add, cap);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_append(const TreeView& tv, const WorkView& wv, const void* k_new,
                           const void* v_new, int n, int dtype, cudaStream_t s,
                           const ProfHook* prof) {

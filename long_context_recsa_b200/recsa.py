@@ -37,6 +37,19 @@ class RecsaConfigC(ctypes.Structure):
     ]
 
 
+class RecsaGatedPoolerC(ctypes.Structure):
+    _fields_ = [
+        ("hidden", ctypes.c_int32),
+        ("tau", ctypes.c_double),
+        ("g", ctypes.c_double),
+        ("rho", ctypes.c_double),
+        ("w", ctypes.c_void_p),
+        ("W1t", ctypes.c_void_p),
+        ("b1", ctypes.c_void_p),
+        ("W2t", ctypes.c_void_p),
+    ]
+
+
 class RecsaTreeInfoC(ctypes.Structure):
     _fields_ = [
         ("n_levels", ctypes.c_int32),
@@ -74,6 +87,7 @@ def _load():
         "recsa_decode_noalloc": [ctypes.POINTER(RecsaConfigC), I64, I32, P, P, ctypes.POINTER(I64),
                                  P, SZ, ctypes.POINTER(I64), P, P, P, P],
         "recsa_probe_bounded_wait": [P, P],
+        "recsa_tree_set_gated_pooler": [P, ctypes.POINTER(RecsaGatedPoolerC)],
         "recsa_tree_free": [P],
         "recsa_status_str": [I32],
     }
@@ -230,6 +244,26 @@ class RecsaTree:
         n = Q.shape[1]
         _check(lib.recsa_prefill_chunk(self.handle, _ptr(Q), pos0, n, _ptr(O), _ptr(sel_out),
                                        _ptr(counts_out), _stream(stream)), "recsa_prefill_chunk")
+
+    def recsa_tree_set_gated_pooler(self, params: dict | None):
+        """Switch the tree's key pooler to Eq.5 (None: back to the stand-in).  params:
+        hidden, tau, g, rho and fp64 device tensors w [d], W1t [2d][h], b1 [h],
+        W2t [h][d]; they must outlive the tree's use of them (kept referenced here)."""
+        if params is None:
+            self._gated = None
+            _check(lib.recsa_tree_set_gated_pooler(self.handle, None), "recsa_tree_set_gated_pooler")
+            return
+        for name in ("w", "W1t", "b1", "W2t"):
+            t = params[name]
+            assert t.dtype == torch.float64 and t.is_cuda and t.is_contiguous(), name
+        p = RecsaGatedPoolerC()
+        p.hidden, p.tau, p.g, p.rho = int(params["hidden"]), float(params["tau"]), \
+            float(params["g"]), float(params["rho"])
+        p.w, p.W1t = params["w"].data_ptr(), params["W1t"].data_ptr()
+        p.b1, p.W2t = params["b1"].data_ptr(), params["W2t"].data_ptr()
+        self._gated = params
+        _check(lib.recsa_tree_set_gated_pooler(self.handle, ctypes.byref(p)),
+               "recsa_tree_set_gated_pooler")
 
     def recsa_get_status(self, stream=None) -> int:
         return lib.recsa_get_status(self.handle, _stream(stream))

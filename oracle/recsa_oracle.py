@@ -31,8 +31,8 @@ Readings where the pages are silent (each also listed in the design notes):
 
 Eq.5 ("Pooler Distillation"): ``gated_pool_keys`` / ``build_tree_gated``, the
 gated key pooler, forward only, with seeded stand-in parameters (its readings are
-listed beside it).  It has no CUDA counterpart yet; its pins are in
-``tests/test_oracle_gated_pooler.py``.
+listed beside it).  Its pins are in ``tests/test_oracle_gated_pooler.py``; the GPU
+path is compared with it in ``tests/test_gpu_gated.py``.
 
 Parity pins: see ``tests/test_oracle_pins.py`` (closed forms for summary values
 and pooled keys, the C*k distance bound, the partition of [0..t] by the
