@@ -393,6 +393,11 @@ def run_ours(args):
             "131K": bench_context(R, I, cfg, 131072, 1, 200, dev, flush, rank),
             "2M": bench_context(R, I, cfg, 2097152, 1, 1000, dev, flush, rank),
         }
+        try:
+            res["contexts"]["2M_level0_in_host_memory"] = bench_offload(R, I, cfg, 2097152, 1, 50,
+                                                                        dev, flush, rank)
+        except (RuntimeError, MemoryError) as e:   # e.g. no room for 8.6 GB of pinned memory
+            res["contexts"]["2M_level0_in_host_memory"] = {"unavailable": str(e)[:200]}
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(K, V, qs, cfg, R)
     if ws > 1:
@@ -667,6 +672,74 @@ def bench_context(R, I, cfg, L, B, steps, dev, flush, rank):
            "timing": "per-step CUDA events around one graph replay (append + decode), "
                      "L2 flushed before every step; the first 3 steps not averaged"}
     del gr, tree, K, V
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_offload(R, I, cfg, L, B, steps, dev, flush, rank):
+    """Decode with level 0 in pinned host memory (the levels above it in HBM): per step
+    the append, the levels >= 1, the gather of each query's level-0 list over the host
+    link into a device staging buffer and level 0 from there, replayed from one
+    captured graph and timed with events.  host_bytes_per_step is what crosses the host
+    link: the level-0 rows of every list (K and V) plus the appended token."""
+    import statistics as st
+    import torch
+    Hq, Hkv, d = W["Hq"], W["Hkv"], W["d"]
+    dt = I.torch_dtype(W["dtype"])
+    cap = L + steps + 16
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank_seed(I.slice_seed(7, I.STREAM_K, 0, 0), rank))
+    Kh = torch.empty(B, Hkv, cap, d, dtype=dt, pin_memory=True)
+    Vh = torch.empty(B, Hkv, cap, d, dtype=dt, pin_memory=True)
+    for h in range(Hkv):   # drawn on the device, copied into the pinned cache
+        Kh[:, h].copy_(torch.randn(B, cap, d, generator=g, device=dev).to(dt))
+        Vh[:, h].copy_(torch.randn(B, cap, d, generator=g, device=dev).to(dt))
+    knew = torch.randn(steps, B, Hkv, 1, d, generator=g, device=dev).to(dt)
+    vnew = torch.randn(steps, B, Hkv, 1, d, generator=g, device=dev).to(dt)
+    qs = torch.randn(steps, B, Hq, d, generator=g, device=dev).to(dt)
+    tree = R.RecsaTree(cfg, cap, B, k0=Kh, v0=Vh)
+    tree.recsa_tree_set_offload_staging()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    tree.recsa_build([L] * B)
+    e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    kst = torch.empty(B, Hkv, 1, d, dtype=dt, device=dev)
+    vst = torch.empty_like(kst)
+    qst = torch.empty(B, Hq, d, dtype=dt, device=dev)
+    out = torch.empty_like(qst)
+    cnt = torch.zeros(B, Hkv, tree.n_sel_levels + 1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gr, stream=stream):
+            tree.recsa_append(kst, vst)
+            tree.recsa_decode(qst, out, None, cnt)
+    torch.cuda.synchronize()
+    times = []
+    for i in range(steps):
+        kst.copy_(knew[i]); vst.copy_(vnew[i]); qst.copy_(qs[i])
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        gr.replay()
+        s1.record()
+        s1.synchronize()
+        times.append(s0.elapsed_time(s1))
+    assert tree.recsa_get_status() == R.RECSA_OK
+    c = cnt.cpu().numpy()
+    host_bytes = int(c[:, :, 0].sum()) * 2 * d * 2 + B * Hkv * 2 * d * 2
+    timed = times[3:]
+    ms = sum(timed) / len(timed)
+    res = {"context": L, "batch": B, "steps": steps, "ms_per_step_median": round(st.median(timed), 4),
+           "ms_per_step_mean": round(ms, 4), "tok_per_s": round(B / (ms / 1e3), 1),
+           "host_bytes_per_step": host_bytes,
+           "host_link_GB_per_s": round(host_bytes / (ms / 1e3) / 1e9, 2),
+           "build_ms_from_host": round(build_ms, 2),
+           "pinned_GB": round(2 * Kh.numel() * Kh.element_size() / 1e9, 2)}
+    del gr, tree, Kh, Vh
     torch.cuda.empty_cache()
     return res
 

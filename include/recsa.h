@@ -293,6 +293,28 @@ typedef struct {
 } recsa_gated_pooler;
 RECSA_API recsa_status recsa_tree_set_gated_pooler(recsa_tree* tree, const recsa_gated_pooler* p);
 
+/* Level 0 in host memory ("Efficiency Results": decode at 1M and 2M tokens with the KV
+ * cache offloaded to the host; "Practical Implications": the levels above 0 are under
+ * 7 % of the cache).  A tree whose k0/v0 passed to recsa_tree_init are pinned host
+ * memory (cudaHostAlloc / cudaMallocHost, mapped into the device address space; they
+ * must both be host or both be device memory, else RECSA_E_INVAL) keeps level 0 there
+ * and its levels >= 1 in the device level tables.  Build and append read and write
+ * level 0 through the host mapping.  recsa_decode then needs a device staging buffer:
+ * after the levels >= 1 have selected S^(1), the rows of each query's level-0 list (the
+ * children of S^(1), Eq.3) are gathered from host memory into it, and level 0 is
+ * attended from there; the result is the same as with level 0 in device memory.
+ * recsa_prefill_chunk returns RECSA_E_UNSUPPORTED on such a tree.
+ *   recsa_offload_staging_bytes: bytes of the staging buffer for `batch` sequences,
+ *     2 * batch * Hkv * C * k * d * element size.
+ *   recsa_tree_set_offload_staging: the caller's device buffer (256-byte aligned, at
+ *     least that many bytes), used by every later decode.  RECSA_E_UNSUPPORTED when
+ *     level 0 is in device memory; a decode on a host-level-0 tree without one returns
+ *     RECSA_E_UNSUPPORTED. */
+RECSA_API recsa_status recsa_offload_staging_bytes(const recsa_config* cfg, int32_t batch,
+                                                   size_t* bytes);
+RECSA_API recsa_status recsa_tree_set_offload_staging(recsa_tree* tree, void* staging,
+                                                      size_t bytes);
+
 /* Free the host handle.  Device memory stays with the caller. */
 RECSA_API recsa_status recsa_tree_free(recsa_tree* tree);
 

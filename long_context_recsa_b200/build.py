@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "librecsa.so")
 SOURCES = ["recsa_api.cu", "tree_kernels.cu", "select_attend.cu", "prefill_tc.cu", "noalloc.cu",
-           "gated.cu"]
+           "gated.cu", "offload.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -71,6 +71,16 @@ extern "C" RECSA_API recsa_status recsa_decode_noalloc(
     if (need > kScratchBytes) return RECSA_E_CAPACITY;   // shape needs more than the fixed scratch
     for (int b = 0; b < batch; ++b)
         if (lengths[b] < 0 || lengths[b] > capacity) return RECSA_E_CAPACITY;
+    {
+        // a level 0 in host memory takes the staged decode of recsa_decode
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, k0) != cudaSuccess) {
+            cudaGetLastError();
+            return RECSA_E_INVAL;
+        }
+        if (a.type == cudaMemoryTypeHost || a.type == cudaMemoryTypeUnregistered)
+            return RECSA_E_UNSUPPORTED;
+    }
     char* scratch = nullptr;
     st = scratch_on_current_device(&scratch);
     if (st != RECSA_OK) return st;

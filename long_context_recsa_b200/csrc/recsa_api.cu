@@ -204,7 +204,35 @@ struct recsa_tree {
     // Eq.5 gated key pooler in place of the stand-in (recsa_tree_set_gated_pooler)
     bool gated;
     GatedView gv;
+    // level 0 in pinned host memory (tv.l0_host): decode stages each query's level-0
+    // list in this device buffer (recsa_tree_set_offload_staging)
+    char* stage;
+    size_t stage_bytes;
+    KVMaps stage_map;
+    bool has_stage_map;
 };
+
+namespace recsa {
+cudaError_t encode_stage_map(const void* base, int64_t rows, int Hkv, int nq, int C, CUtensorMap* m);
+}  // namespace recsa
+
+// Where a level-0 buffer lives: 1 pinned host memory (its device address in *dev),
+// 0 device memory, -1 memory the GPU cannot read (pageable host memory).
+static int level0_residence(const void* p, const void** dev) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    if (a.type == cudaMemoryTypeHost) {
+        if (!a.devicePointer) return -1;
+        *dev = a.devicePointer;
+        return 1;
+    }
+    if (a.type == cudaMemoryTypeUnregistered) return -1;
+    *dev = p;
+    return 0;
+}
 
 // Runs a pending ancestor re-pooling on `stream` (before a call that needs the
 // complete tree).
@@ -268,6 +296,9 @@ recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t 
     if (sb % per16 || sh % per16 || stt % per16) return RECSA_E_INVAL;
     if (level_bytes < L.level_bytes || workspace_bytes < L.ws_bytes) return RECSA_E_CAPACITY;
 
+    const void *k0d = nullptr, *v0d = nullptr;
+    const int rk = level0_residence(k0, &k0d), rv = level0_residence(v0, &v0d);
+    if (rk < 0 || rv < 0 || rk != rv) return RECSA_E_INVAL;
     recsa_tree* t = (recsa_tree*)calloc(1, sizeof(recsa_tree));
     if (!t) return RECSA_E_INVAL;
     t->cfg = *cfg;
@@ -276,7 +307,8 @@ recsa_status recsa_tree_init(const recsa_config* cfg, int64_t capacity, int32_t 
     t->B = batch;
     t->Qmax = max_queries;
     TreeView& tv = t->tv;
-    tv.k0 = k0; tv.v0 = v0; tv.k0w = k0; tv.v0w = v0;
+    tv.k0 = k0d; tv.v0 = v0d; tv.k0w = const_cast<void*>(k0d); tv.v0w = const_cast<void*>(v0d);
+    tv.l0_host = rk;
     tv.s_b = sb; tv.s_h = sh; tv.s_t = stt;
     tv.levels = (char*)levels;
     for (int l = 0; l < kMaxLevels; ++l) {
@@ -401,8 +433,34 @@ recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_
     qv.q_begin = 0;
     qv.nq = t->B;
     qv.walk = t->walk_pending ? 1 : 0;
+    const cudaStream_t s = (cudaStream_t)stream;
+    if (t->tv.l0_host) {
+        // level 0 in host memory: levels >= 1, the gather of each query's level-0 list
+        // into the staging buffer, then level 0 from there and the merge
+        if (!t->stage) return RECSA_E_UNSUPPORTED;
+        const size_t half = t->stage_bytes / 2;
+        qv.phase = 1;
+        cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof,
+                                             t->has_maps ? t->maps : nullptr);
+        if (e == cudaSuccess)
+            e = launch_gather_level0(t->tv, t->wv, qv, t->stage, t->stage + half, t->cfg.dtype, s);
+        if (e != cudaSuccess) return RECSA_E_CUDA;
+        t->walk_pending = false;
+        qv.phase = 2;
+        qv.walk = 0;
+        qv.l0k = t->stage;
+        qv.l0v = t->stage + half;
+        KVMaps m2[kMaxLevels];
+        const bool sw = t->has_maps && t->has_stage_map;
+        if (sw) {
+            memcpy(m2, t->maps, sizeof(m2));
+            m2[0] = t->stage_map;
+        }
+        e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof, sw ? m2 : nullptr);
+        return e == cudaSuccess ? RECSA_OK : RECSA_E_CUDA;
+    }
     cudaError_t e =
-        launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, (cudaStream_t)stream, &t->prof,
+        launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof,
                              t->has_maps ? t->maps : nullptr);
     if (e != cudaSuccess) return RECSA_E_CUDA;
     t->walk_pending = false;
@@ -428,6 +486,7 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
                                  int32_t* sel_out, int32_t* counts_out, void* stream) {
     if (!t || !Q || !O || n < 1 || pos0 < 0) return RECSA_E_INVAL;
     if (!aligned16(Q) || !aligned16(O)) return RECSA_E_INVAL;
+    if (t->tv.l0_host) return RECSA_E_UNSUPPORTED;   // offloaded level 0: decode only
     for (int b = 0; b < t->B; ++b)
         if (pos0 + n > t->host_len[b]) return RECSA_E_CAPACITY;
     const cudaStream_t s = (cudaStream_t)stream;
@@ -478,6 +537,40 @@ recsa_status recsa_prefill_chunk(recsa_tree* t, const void* Q, int64_t pos0, int
         cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof,
                                                      t->has_maps ? t->maps : nullptr);
         if (e != cudaSuccess) return RECSA_E_CUDA;
+    }
+    return RECSA_OK;
+}
+
+recsa_status recsa_offload_staging_bytes(const recsa_config* cfg, int32_t batch, size_t* bytes) {
+    recsa_status st = check_config(cfg);
+    if (st != RECSA_OK) return st;
+    if (!bytes || batch < 1 || batch > RECSA_MAX_BATCH) return RECSA_E_INVAL;
+    const size_t es = cfg->dtype == RECSA_BF16 ? 2 : 4;
+    *bytes = 2 * (size_t)batch * cfg->n_kv_heads * (size_t)cfg->C * cfg->k * cfg->head_dim * es;
+    return RECSA_OK;
+}
+
+recsa_status recsa_tree_set_offload_staging(recsa_tree* t, void* staging, size_t bytes) {
+    if (!t) return RECSA_E_INVAL;
+    if (!t->tv.l0_host) return RECSA_E_UNSUPPORTED;   // level 0 is already in device memory
+    size_t need = 0;
+    recsa_status st = recsa_offload_staging_bytes(&t->cfg, t->B, &need);
+    if (st != RECSA_OK) return st;
+    if (!staging || ((uintptr_t)staging & 255u)) return RECSA_E_INVAL;
+    if (bytes < need) return RECSA_E_CAPACITY;
+    const void* d = nullptr;
+    if (level0_residence(staging, &d) != 0) return RECSA_E_INVAL;   // must be device memory
+    t->stage = (char*)staging;
+    t->stage_bytes = need;
+    t->has_stage_map = false;
+    if (t->has_maps) {
+        const size_t half = need / 2;
+        t->has_stage_map =
+            encode_stage_map(t->stage, t->wv.ck, t->tv.Hkv, t->B, t->tv.C, &t->stage_map.k) ==
+                cudaSuccess &&
+            encode_stage_map(t->stage + half, t->wv.ck, t->tv.Hkv, t->B, t->tv.C,
+                             &t->stage_map.v) == cudaSuccess;
+        if (!t->has_stage_map) return RECSA_E_CUDA;
     }
     return RECSA_OK;
 }
@@ -627,9 +720,19 @@ static cudaError_t encode_table(CUtensorMap* m, const void* base, int64_t rows, 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_stage_map(const void* base, int64_t rows, int Hkv, int nq, int C, CUtensorMap* m) {
+    return encode_table(m, base, rows, Hkv, nq, 256, rows * 256, rows * 256 * Hkv, C);
+}
+
 cudaError_t encode_kv_maps(const TreeView& tv, KVMaps* maps) {
     for (int l = 0; l < tv.n_levels && l < kMaxLevels; ++l) {
         cudaError_t e;
+        if (l == 0 && tv.l0_host) {
+            // a host-resident level 0 is never staged by TMA (decode stages it through
+            // the gather into a device buffer with its own map)
+            memset(&maps[0], 0, sizeof(maps[0]));
+            continue;
+        }
         if (l == 0) {
             const int64_t es = 2;
             e = encode_table(&maps[0].k, tv.k0, tv.cap, tv.Hkv, tv.B, tv.s_t * es, tv.s_h * es,

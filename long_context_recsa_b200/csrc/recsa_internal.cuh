@@ -37,6 +37,8 @@ struct TreeView {
     float scale;
     double rope_base;
     float w[RECSA_MAX_C];      // pooler logits; kernels form softmax(w[0..m-1]) in fp64
+    int l0_host;               // level 0 lives in pinned host memory: plain loads and
+                               // stores only (no TMA copy or bulk prefetch touches it)
 };
 
 // Parameters of the Eq.5 gated key pooler (caller-owned fp64 device arrays).
@@ -70,6 +72,14 @@ struct QueryView {
     // decode only: the level-0 launch also re-pools the ancestors of each sequence's
     // newest token (extra CTAs after the attention CTAs)
     int walk;
+    // decode with level 0 in host memory, in two launches around a gather:
+    //   phase 1: levels >= 1 only (no level 0, no merge);
+    //   phase 2: level 0 only, read from the staging copy l0k/l0v [nq][Hkv][C*k][D]
+    //            in list order (entry j at row j), then the merge;
+    //   phase 0: every level and the merge (level 0 read where it lives).
+    int phase;
+    const void* l0k;
+    const void* l0v;
 };
 
 // TMA tensor maps of one level's K and V tables (bf16, d = 128): 4-d (d, row, KV
@@ -382,6 +392,11 @@ inline bool uses_kv_maps(int dtype, int D, int C) {
 cudaError_t encode_kv_maps(const TreeView& tv, KVMaps* maps);
 cudaError_t prepare_tree_kernels(const TreeView& tv, int dtype);
 cudaError_t launch_set_lengths(const WorkView& wv, const int64_t* lengths, int B, cudaStream_t s);
+// The level-0 list of every decode query, copied in list order from the level-0 cache
+// (host memory) into the staging buffer [nq][Hkv][C*k][D] (K and V), after a phase-1
+// pass has selected level 1 (offload.cu).
+cudaError_t launch_gather_level0(const TreeView& tv, const WorkView& wv, const QueryView& qv,
+                                 void* stage_k, void* stage_v, int dtype, cudaStream_t s);
 // Eq.5 levels 1.. with the gated key pooler: every node (add == 0) or the nodes
 // covering the `add` tokens appended at the device-side lengths (gated.cu).
 cudaError_t launch_gated_levels(const TreeView& tv, const WorkView& wv, const GatedView& gv,

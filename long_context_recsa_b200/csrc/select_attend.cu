@@ -1397,6 +1397,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int level = NL; level >= 0; --level) {
         const bool L0 = level == 0;
         if (level > lstar) continue;   // not scored: recorded after the pass
+        if (qv.phase == 2 && !L0) continue;   // levels >= 1 were done by the phase-1 launch
+        if (qv.phase == 1 && L0) break;       // level 0 and the merge: the phase-2 launch
         if (level < lstar) {
             // the parent list S^(level+1): every CTA of the cluster has stored the
             // entries this CTA needs into its par_next; after the barrier they are in
@@ -1420,14 +1422,20 @@ __global__ void __launch_bounds__(kThreads, 2)
             pdl_launch_dependents();   // the next kernel may start launching
         }
         const int nA = list_size(t, lstar, level, C, lgC, k);
-        const bool identity = level == lstar;
+        // phase 2 reads level 0 from the staging copy, where entry j is row j
+        const bool identity = level == lstar || qv.phase == 2;
         const int npar_all = cdiv(nA + C - 1, C, lgC);
         const int chunk = ((npar_all + nsplit - 1) / nsplit) * C;
         const int j0 = split * chunk;
         const int j1 = min(nA, j0 + chunk);
         const T *kbase, *vbase;
         int64_t rs;
-        if (L0) {
+        if (L0 && qv.phase == 2) {
+            const int64_t so = ((int64_t)qloc * tv.Hkv + kvh) * (int64_t)wv.ck * D;
+            kbase = reinterpret_cast<const T*>(qv.l0k) + so;
+            vbase = reinterpret_cast<const T*>(qv.l0v) + so;
+            rs = D;
+        } else if (L0) {
             kbase = reinterpret_cast<const T*>(tv.k0) + (b * tv.s_b + kvh * tv.s_h);
             vbase = reinterpret_cast<const T*>(tv.v0) + (b * tv.s_b + kvh * tv.s_h);
             rs = tv.s_t;
@@ -1629,7 +1637,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!L0) cluster_wait();   // matches the arrive after this CTA's remote reads
     }
 
-    if (split == 0) {
+    if (split == 0 && qv.phase != 2) {
         // the levels above the first scored one: their whole lists are selected
         for (int l = lstar + 1; l <= NL; ++l) {
             if (qv.sel_out)
@@ -1640,6 +1648,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (cnt_usr) cnt_usr[l] = 0;
             }
         }
+    }
+    if (qv.phase == 1) {
+        // the peers' parent-list stores into this CTA's shared memory have landed
+        // before any CTA of the cluster exits
+        pdl_launch_dependents();
+        cluster.sync();
+        return;
     }
     // every partial of the unit is written: merge them, this CTA taking a slice of
     // the G output heads

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256, 2) build_pass_kernel(TreeView tv, WorkVie
         const int m = (int)imin64(C, n_s - i1 * C);
         // rows of the parent two steps ahead go to L2 while this one is pooled
         const int64_t ia = i1 + 2;
-        if (lane == 0 && c1 + 2 < C && ia < n_s1) {
+        if (lane == 0 && c1 + 2 < C && ia < n_s1 && !(s == 0 && tv.l0_host)) {
             const int ma = (int)imin64(C, n_s - ia * C);
             if (rs == D) {
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sk + ia * C * rs),

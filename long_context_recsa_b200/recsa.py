@@ -88,6 +88,8 @@ def _load():
                                  P, SZ, ctypes.POINTER(I64), P, P, P, P],
         "recsa_probe_bounded_wait": [P, P],
         "recsa_tree_set_gated_pooler": [P, ctypes.POINTER(RecsaGatedPoolerC)],
+        "recsa_offload_staging_bytes": [ctypes.POINTER(RecsaConfigC), I32, ctypes.POINTER(SZ)],
+        "recsa_tree_set_offload_staging": [P, P, SZ],
         "recsa_tree_free": [P],
         "recsa_status_str": [I32],
     }
@@ -264,6 +266,19 @@ class RecsaTree:
         self._gated = params
         _check(lib.recsa_tree_set_gated_pooler(self.handle, ctypes.byref(p)),
                "recsa_tree_set_gated_pooler")
+
+    def recsa_tree_set_offload_staging(self, staging: torch.Tensor | None = None):
+        """Give a tree whose level 0 is in pinned host memory its device staging
+        buffer (allocated here when not given; kept referenced)."""
+        if staging is None:
+            nb = ctypes.c_size_t()
+            c = self.cfg.to_c()
+            _check(lib.recsa_offload_staging_bytes(ctypes.byref(c), self.batch, ctypes.byref(nb)),
+                   "recsa_offload_staging_bytes")
+            staging = torch.empty(nb.value, dtype=torch.uint8, device="cuda")
+        self._staging = staging
+        _check(lib.recsa_tree_set_offload_staging(self.handle, _ptr(staging), staging.numel()),
+               "recsa_tree_set_offload_staging")
 
     def recsa_get_status(self, stream=None) -> int:
         return lib.recsa_get_status(self.handle, _stream(stream))
