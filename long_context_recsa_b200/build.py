@@ -34,22 +34,32 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+OUT_BOUNDS = os.path.join(HERE, "librecsa_bounds.so")
+
+
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
+    """Compile the library (librecsa.so), or with debug_bounds the bounds-checked
+    variant (librecsa_bounds.so: every gather row and selection rank is range-checked
+    on the device and a failure is recorded in the status word)."""
+    out = OUT_BOUNDS if debug_bounds else OUT
     deps = [os.path.join(CSRC, s) for s in SOURCES]
     deps += [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
     deps.append(os.path.join(HERE, "..", "include", "recsa.h"))
-    if not force and not _stale(OUT, deps):
-        return OUT
+    if not force and not _stale(out, deps):
+        return out
     cmd = [nvcc_path(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           "-o", OUT + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
+           "-o", out + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
+    if debug_bounds:
+        cmd.insert(1, "-DRECSA_DEBUG_BOUNDS")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(OUT + ".tmp", OUT)
-    return OUT
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                debug_bounds="--bounds" in sys.argv))

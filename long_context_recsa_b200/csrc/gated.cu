@@ -233,6 +233,7 @@ static cudaError_t gated_levels_impl(const TreeView& tv, const WorkView& wv, con
     int64_t grid = (work + kGatedWarps - 1) / kGatedWarps;
     if (grid > nsm) grid = nsm;
     if (grid < 1) grid = 1;
+    NvtxRange nv(add == 0 ? "recsa build (gated pooler)" : "recsa append levels (gated pooler)");
     for (int lvl = 1; lvl < tv.n_levels; ++lvl) {
         gated_level_kernel<T, D><<<(unsigned)grid, kGatedWarps * 32, sm, s>>>(tv, wv, gv, lvl, add);
         e = cudaGetLastError();

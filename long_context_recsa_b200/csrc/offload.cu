@@ -34,8 +34,9 @@ __global__ void __launch_bounds__(256) gather_level0_kernel(TreeView tv, WorkVie
     for (int j = blockIdx.x * RPB + tr; j < n0; j += gridDim.x * RPB) {
         // entry j of A^(0): token j when level 0 is the first scored level, else child
         // j mod C of the (j / C)-th node of S^(1)
-        const int64_t tok = lstar == 0 ? (int64_t)j
-                                       : (int64_t)C * S1[cdiv(j, C, lgC)] + cmod(j, C, lgC);
+        int64_t tok = lstar == 0 ? (int64_t)j
+                                 : (int64_t)C * S1[cdiv(j, C, lgC)] + cmod(j, C, lgC);
+        if (!in_bounds(tok >= 0 && tok <= t, wv.status)) tok = 0;
         const uint4 kx = *reinterpret_cast<const uint4*>(k0 + tok * tv.s_t + tc * VEC);
         const uint4 vx = *reinterpret_cast<const uint4*>(v0 + tok * tv.s_t + tc * VEC);
         *reinterpret_cast<uint4*>(stage_k + so + (int64_t)j * D + tc * VEC) = kx;
@@ -46,6 +47,7 @@ __global__ void __launch_bounds__(256) gather_level0_kernel(TreeView tv, WorkVie
 template <typename T, int D>
 static cudaError_t gather_impl(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                void* sk, void* sv, cudaStream_t s) {
+    NvtxRange nv("recsa gather level 0");
     const unsigned slices = (unsigned)((wv.ck + 255) / 256);
     dim3 grid(slices < 8 ? slices : 8, (unsigned)(qv.nq * tv.Hkv));
     gather_level0_kernel<T, D><<<grid, 256, 0, s>>>(tv, wv, qv, reinterpret_cast<T*>(sk),

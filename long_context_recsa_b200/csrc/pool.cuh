@@ -210,7 +210,7 @@ __device__ __forceinline__ void level_rows(const TreeView& tv, int l, int b, int
 // RB: children rows loaded per batch (fewer registers inside a larger kernel).
 template <typename T, int D, int RB = 16>
 __device__ __forceinline__ void ancestor_walk(const TreeView& tv, int b, int h, int64_t t,
-                                              double* pre, const double* alpha) {
+                                              double* pre, const double* alpha, uint32_t* status) {
     constexpr int N = PoolShape<T, D>::DPL;
     const int C = tv.C, lgC = tv.lgC;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -221,8 +221,9 @@ __device__ __forceinline__ void ancestor_walk(const TreeView& tv, int b, int h, 
     for (int l = 1 + warp; l <= nl; l += nwarps) {
         int64_t x = t;   // ancestor index at level l-1
         for (int j = 1; j < l; ++j) x = cdiv64(x, C, lgC);
-        const int64_t i = cdiv64(x, C, lgC);
-        const int m = (int)(x - i * C) + 1;
+        int64_t i = cdiv64(x, C, lgC);
+        int m = (int)(x - i * C) + 1;
+        if (!in_bounds(i >= 0 && x < tv.rows[l - 1] && i < tv.rows[l], status)) { i = 0; m = 1; }
         const T *sk, *sv;
         int64_t rs;
         level_rows<T>(tv, l - 1, b, h, sk, sv, rs);

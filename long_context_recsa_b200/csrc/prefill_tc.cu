@@ -372,6 +372,7 @@ static cudaError_t prefill_top_impl(const TreeView& tv, const WorkView& wv, cons
 cudaError_t launch_prefill_top_tc(const TreeView& tv, const WorkView& wv, const QueryView& qv,
                                   const TcView& tc, int lt, int64_t a_max, int dtype, cudaStream_t s,
                                   const ProfHook* prof) {
+    NvtxRange nv("recsa prefill top-level product");
 #define RECSA_TC_G(T, D)                                                       \
     do {                                                                       \
         if (tv.G == 1) return prefill_top_impl<T, D, 1>(tv, wv, qv, tc, lt, a_max, s, prof); \

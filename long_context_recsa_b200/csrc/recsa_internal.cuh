@@ -4,6 +4,7 @@
 #include <cuda.h>   // CUtensorMap only; maps are encoded through the runtime's driver entry point
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "../../include/recsa.h"
@@ -17,7 +18,14 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // Device status word values (first error wins).
 enum : uint32_t { kStatusOk = 0, kStatusBadQuery = 1, kStatusCapacity = 2, kStatusTimeout = 3,
-                  kStatusLayout = 4 /* a staging buffer was misaligned */ };
+                  kStatusLayout = 4 /* a staging buffer was misaligned */,
+                  kStatusBounds = 5 /* a range check of the bounds-checked build failed */ };
+
+// Named range around each launch for profilers (NVTX; no cost without a tool).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 // Location of the tree in device memory.
 struct TreeView {
@@ -127,6 +135,19 @@ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ?
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t code) {
     atomicCAS(st, 0u, code);
 }
+
+// Range checks of the bounds-checked build (-DRECSA_DEBUG_BOUNDS): a row or rank index
+// about to be used for a gather or a store.  A failed check records kStatusBounds (the
+// caller then falls back to an index that is in range); without the flag the check
+// compiles to true.
+#ifdef RECSA_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t* st) {
+    if (!ok) set_status(st, kStatusBounds);
+    return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, uint32_t*) { return true; }
+#endif
 
 template <typename T> struct VecOf;
 template <> struct VecOf<float> { static constexpr int N = 4; };

@@ -1268,7 +1268,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int b = ci / tv.Hkv, h = ci % tv.Hkv;
         const int64_t t = wv.lens[b] - 1;
         __syncthreads();
-        if (t >= 1) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha);
+        if (t >= 1) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha, wv.status);
         return;
     }
     constexpr int kRow = D * (int)sizeof(T);
@@ -1491,8 +1491,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int nk = pre ? 0 : nw;   // blocks [0, nk) are K, [nk, nk + nw) are V
         const WarpRing R{ring + (size_t)warp * nsw * slot_bytes, bars + warp * nsw, nsw,
                          slot_bytes, wv.status, misc + kMiscFailed};
+        // rows of the table this level reads (the staging copy in phase 2)
+        const int64_t trows = L0 ? (qv.phase == 2 ? (int64_t)wv.ck : tv.cap) : tv.rows[level];
         auto group_first = [&](int jb) -> int64_t {
-            return identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
+            const int64_t f = identity ? (int64_t)jb : (int64_t)C * par[cdiv(jb, C, lgC)];
+            return in_bounds(f >= 0 && f < trows && jb >= 0 && jb < nA, wv.status) ? f : 0;
         };
         const KVMaps* lmap = &maps.m[level < kMapLevels ? level : 0];
         auto issue = [&](int q) {
@@ -1550,6 +1553,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             cluster_wait();   // every CTA's zeroed histograms (and keys) are in place
             // 2. exact top-(k-1) over all M keys; this CTA writes S for its entries
             auto mark = [&](int i, int r) {
+                if (!in_bounds(r >= 0 && r < K1 && i >= j0 && i < j0 + n_sc &&
+                               r / ppc_next < nsplit, wv.status))
+                    return;
                 const int node = nodes[i - j0];
                 sel_ws[r] = node;
                 if (sel_usr) sel_usr[r] = node;
@@ -1735,6 +1741,8 @@ static cudaError_t select_attend_variant(const TreeView& tv, const WorkView& wv,
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     prof_mark(prof, 0, true, s);
+    NvtxRange nv(qv.phase == 1 ? "recsa pass (levels >= 1)" : qv.phase == 2 ? "recsa pass (level 0)"
+                 : "recsa pass");
     cudaError_t e = cudaLaunchKernelEx(&cfg, pass_kernel<T, D, G, SW>, tv, wv, qv, pm, CH, NA, nsw);
     prof_mark(prof, 0, false, s);
     if (e != cudaSuccess) return e;

@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(256) append_walk_kernel(TreeView tv, WorkView 
     const int64_t t = wv.lens[b] - 1;
     __syncthreads();
     if (t < 1) return;
-    ancestor_walk<T, D>(tv, b, h, t, pre, alpha);
+    ancestor_walk<T, D>(tv, b, h, t, pre, alpha, wv.status);
 }
 
 // Waits on an mbarrier that nothing arrives on, through the bounded wait of every
@@ -232,6 +232,7 @@ cudaError_t launch_bounded_wait_probe(uint32_t* status, cudaStream_t s) {
 // ----------------------------------------------------------------------------
 template <typename T, int D>
 static cudaError_t run_passes(const TreeView& tv, const WorkView& wv, int64_t add, cudaStream_t s) {
+    NvtxRange nv(add == 0 ? "recsa build" : "recsa append levels");
     for (int src = 0; src + 1 < tv.n_levels; src += 2) {
         int64_t span2 = 1;
         for (int i = 0; i < src + 2; ++i) span2 *= tv.C;
@@ -286,6 +287,7 @@ static cudaError_t append_token_impl(const TreeView& tv, const WorkView& wv, con
     cudaLaunchAttribute attr[1] = {pdl_attribute()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    NvtxRange nv("recsa append token");
     prof_mark(prof, -1, true, s);
     cudaError_t e = cudaLaunchKernelEx(&cfg, append_token_kernel<T, D>, tv, wv,
                                        reinterpret_cast<const T*>(k_new),
@@ -305,6 +307,7 @@ static cudaError_t append_walk_impl(const TreeView& tv, const WorkView& wv, cuda
     cudaLaunchAttribute attr[1] = {pdl_attribute()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    NvtxRange nv("recsa ancestor walk");
     cudaError_t e = cudaLaunchKernelEx(&cfg, append_walk_kernel<T, D>, tv, wv);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -66,9 +66,12 @@ class RecsaTreeInfoC(ctypes.Structure):
 
 
 def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"librecsa.so not built ({LIB_PATH}); run python -m long_context_recsa_b200.build")
-    lib = ctypes.CDLL(LIB_PATH)
+    # RECSA_LIBRARY selects another build of this library (the bounds-checked
+    # librecsa_bounds.so in its tests); there is no fallback when it is missing
+    path = os.environ.get("RECSA_LIBRARY", LIB_PATH)
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not built; run python -m long_context_recsa_b200.build")
+    lib = ctypes.CDLL(path)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     sig = {
         "recsa_query_sizes": [ctypes.POINTER(RecsaConfigC), I64, I32, I32, ctypes.POINTER(SZ),

@@ -147,3 +147,65 @@ def test_decode_2m_with_append_sampled_unit(R):
     assert tree.recsa_get_status() == R.RECSA_OK
     check_unit(R, tree, K, V, q[0, 2 * G:3 * G], 0, 2, L + 1, L, w,
                sel[0, 2].cpu().numpy(), cnt[0, 2].cpu().numpy(), out[0, 2 * G:3 * G])
+
+
+def test_captured_decode_graph_long_replay_524k(R):
+    """The bench's timed path: one captured append + decode graph replayed 120 times
+    at L = 524288 (device-side lengths advance, the appended tokens' ancestors are
+    re-pooled by the pass kernel's extra CTAs).  Replays 0, 1, 60 and 119 of two units
+    are checked against the oracle, which is built once over the final length: for a
+    query at t every listed node other than the current one covers tokens <= t only,
+    and the current node is never scored nor a summary.  The final trees bit for bit."""
+    L0, reps = 524288, 120
+    checks = (0, 1, 60, reps - 1)
+    units = (0, 5)
+    w = H.w_for(C)
+    cap = L0 + reps + 16
+    K, V, _ = device_inputs(7, 1, cap, [L0 + reps])
+    Q = I.q_rows(7, 0, reps, Hq, d, "bf16", device="cuda")
+    Kb, Vb = K.clone(), V.clone()
+    Kb[:, :, L0:] = 0
+    Vb[:, :, L0:] = 0
+    tree = R.RecsaTree(cfg_for(R, w), cap, 1, k0=Kb, v0=Vb)
+    tree.recsa_build([L0])
+    kst = torch.empty(1, Hkv, 1, d, dtype=torch.bfloat16, device="cuda")
+    vst, qst = torch.empty_like(kst), torch.empty(1, Hq, d, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(qst)
+    nl = tree.n_sel_levels
+    sel = torch.empty(1, Hkv, nl, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, Hkv, nl + 1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gr, stream=stream):
+            tree.recsa_append(kst, vst)
+            tree.recsa_decode(qst, out, sel, cnt)
+    torch.cuda.synchronize()
+    got = {}
+    for r in range(reps):
+        kst.copy_(K[:, :, L0 + r:L0 + r + 1])
+        vst.copy_(V[:, :, L0 + r:L0 + r + 1])
+        qst.copy_(Q[r:r + 1])
+        gr.replay()
+        if r in checks:
+            torch.cuda.synchronize()
+            got[r] = (out.clone(), sel.cpu().numpy(), cnt.cpu().numpy())
+    torch.cuda.synchronize()
+    del gr
+    assert tree.recsa_get_status() == R.RECSA_OK
+    # the host copy of the lengths saw the captured append once; replays advance only
+    # the device-side lengths
+    assert tree.host_lengths() == [L0 + 1]
+    from oracle import recsa_oracle as O_
+    for h in units:
+        levels = O_.build_tree(H.to64(K[0, h, :L0 + reps]), H.to64(V[0, h, :L0 + reps]), C,
+                               np.asarray(w, dtype=np.float64), "bf16")
+        H.compare_tree(tree, levels, 0, h, "bf16")
+        for r in checks:
+            t = L0 + r
+            qg = H.to64(Q[r, h * G:(h + 1) * G])
+            res = O_.select_and_attend(levels, qg, t, C, k, base=1e6)
+            o, sl, cn = got[r]
+            cur = H.check_selection(levels, qg, t, C, k, 1e6, res, sl[0, h], cn[0, h], nl)
+            err = H.max_abs(H.to64(o[0, h * G:(h + 1) * G]), cur.out)
+            assert err <= H.TOL_OUT["bf16"], f"replay {r} head {h}: output max-abs {err}"

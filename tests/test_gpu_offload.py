@@ -66,9 +66,14 @@ def test_offloaded_decode_equals_device_decode(R, dtype, d, C, k, G):
             vn = V[:, :, 5000 + s:5000 + s + 1].contiguous()
             dev.recsa_append(kn, vn)
             host.recsa_append(kn, vn)
-    for lvl in range(1, dev.n_levels):
-        assert torch.equal(dev.level_tables(lvl)[0], host.level_tables(lvl)[0]), f"K level {lvl}"
-        assert torch.equal(dev.level_tables(lvl)[1], host.level_tables(lvl)[1]), f"V level {lvl}"
+    for lvl in range(1, dev.n_levels):   # the rows each sequence's tree holds
+        for b in range(B):
+            n = -(-(lengths[b] + steps) // C ** lvl)
+            if -(-(lengths[b] + steps) // C ** (lvl - 1)) <= 1:
+                continue   # the level below is already this sequence's root
+            for i in (0, 1):
+                assert torch.equal(dev.level_tables(lvl)[i][b, :, :n],
+                                   host.level_tables(lvl)[i][b, :, :n]), f"level {lvl} seq {b}"
     with pytest.raises(R.RecsaError) as e:
         host.prefill(q[:, :2].contiguous(), 100)
     assert e.value.status == R.RECSA_E_UNSUPPORTED
