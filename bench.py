@@ -32,11 +32,11 @@ METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
 # capture at batch 1 (the pass kernel's summary under profiles/); a launch covers
 # batch x 8 independent units, so the batch-B figure is B times this.  Valid only
 # for the kernel sources it was taken from: any edit to them turns it into null.
-TRAFFIC_PASS_B1 = {"bytes": 44_201_728 + 149_504,
+TRAFFIC_PASS_B1 = {"bytes": 44_192_768 + 109_312,
                    "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
                                "long_context_recsa_b200/csrc/recsa_internal.cuh",
                                "long_context_recsa_b200/csrc/pool.cuh"],
-                   "sha256": "c241b4a737f4525f8e07d150c3d882357917f2c18e17851d3510d574f79065e4"}
+                   "sha256": "b995fc588e836240cb2430bc4c2fe9a68d13e0a8a27651aac9a75a54052db134"}
 
 
 def captured_traffic(kernel: str, batch: int):
@@ -579,7 +579,7 @@ def prefill_roofline(R, pt, Q, pos0, O, dev):
             "note": "logical bytes are the lists' reads; most hit L2 (rows share the tree)"}
 
 
-def bench_gated_build(R, I, cfg, K, V, cap, B, L, dev, hidden=64):
+def bench_gated_build(R, I, cfg, K, V, cap, B, L, dev, hidden=32):
     """The same tree built with the Eq.5 gated key pooler (seeded parameters, MLP
     width `hidden`), timed with events: fp64 per-node statistics and MLP, one warp
     per node."""

@@ -20,15 +20,15 @@
 
 namespace recsa {
 
-constexpr int kGatedWarps = 4;   // warps per CTA (shared memory holds the fp64 weights)
-
-// Shared memory: w [D], W1t [2D][h], b1 [h], W2t [h][D], then per warp z [2D],
-// mu [D], pm [D], hid [h], alpha [C].
-inline size_t gated_smem(int D, int h, int C) {
+// Shared memory of a CTA of `warps` warps: w [D], W1t [2D][h], b1 [h], W2t [h][D],
+// then per warp z [2D], mu [D], pm [D], hid [h], alpha [C].
+inline size_t gated_smem(int D, int h, int warps) {
     const size_t weights = (size_t)D + 2 * (size_t)D * h + h + (size_t)h * D;
     const size_t per_warp = 4 * (size_t)D + h + RECSA_MAX_C;
-    return sizeof(double) * (weights + kGatedWarps * per_warp);
+    return sizeof(double) * (weights + warps * per_warp);
 }
+// Warps per CTA: 8 when their scratch fits beside the weights, else 4.
+inline int gated_warps(int D, int h) { return gated_smem(D, h, 8) <= 227 * 1024 ? 8 : 4; }
 
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
@@ -93,17 +93,21 @@ __device__ void gated_pool_node(const T* sk, const T* sv, int64_t rs, int m, con
     ss = warp_sum_f64(ss);
     const double sigma = sqrt(ss / (dm * (double)D) + 1e-6);
     __syncwarp();
-    // 3. softmax over the children of tau * projection / sigma
+    // 3. softmax over the children of tau * projection / sigma: lane c < m forms
+    //    exp(logit_c - max) once; the sum is taken in child order
     double mx = -INFINITY;
     for (int c = 0; c < m; ++c) mx = fmax(mx, gv.tau * al[c] / sigma);
+    __syncwarp();
+    for (int c = lane; c < m; c += 32) al[c] = exp(gv.tau * al[c] / sigma - mx);
+    __syncwarp();
     double sum = 0.0;
-    for (int c = 0; c < m; ++c) sum += exp(gv.tau * al[c] / sigma - mx);
+    for (int c = 0; c < m; ++c) sum += al[c];
     // 4. p = sum_c alpha_c x_c
     double p[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) p[e] = 0.0;
     for (int c = 0; c < m; ++c) {
-        const double a = exp(gv.tau * al[c] / sigma - mx) / sum;
+        const double a = al[c] / sum;
         double x[N];
         load_dims<T, N>(sk + c * rs, off, x);
 #pragma unroll
@@ -155,7 +159,7 @@ __device__ void gated_pool_node(const T* sk, const T* sv, int64_t rs, int m, con
 // length L_old) or every node of [0, L) (add == 0).  A persistent grid: each CTA
 // stages the weights once and its warps take nodes in turn.
 template <typename T, int D>
-__global__ void __launch_bounds__(kGatedWarps * 32, 1)
+__global__ void __launch_bounds__(256, 1)
     gated_level_kernel(TreeView tv, WorkView wv, GatedView gv, int lvl, int64_t add) {
     extern __shared__ __align__(16) double gsm[];
     const int h = gv.h;
@@ -170,6 +174,7 @@ __global__ void __launch_bounds__(kGatedWarps * 32, 1)
     for (int i = threadIdx.x; i < h * D; i += blockDim.x) W2t[i] = gv.W2t[i];
     __syncthreads();
     const int warp = threadIdx.x >> 5;
+    const int nwarp_cta = blockDim.x >> 5;
     double* z = scratch + warp * (4 * D + h + RECSA_MAX_C);
     double* mu_s = z + 2 * D;
     double* pm_s = mu_s + D;
@@ -181,8 +186,8 @@ __global__ void __launch_bounds__(kGatedWarps * 32, 1)
     const int64_t span_c = span / C;   // tokens per child
     // work items: (b, h, node) over all (sequence, KV head) units, node in [p_lo, p_hi]
     const int nbh = tv.B * tv.Hkv;
-    const int64_t gw = (int64_t)blockIdx.x * kGatedWarps + warp;
-    const int64_t nwarps = (int64_t)gridDim.x * kGatedWarps;
+    const int64_t gw = (int64_t)blockIdx.x * nwarp_cta + warp;
+    const int64_t nwarps = (int64_t)gridDim.x * nwarp_cta;
     // per unit, the number of nodes to pool at this level; the units are taken in
     // order, each warp stepping through the flattened (unit, node) space
     int64_t base = 0;
@@ -220,7 +225,8 @@ __global__ void __launch_bounds__(kGatedWarps * 32, 1)
 template <typename T, int D>
 static cudaError_t gated_levels_impl(const TreeView& tv, const WorkView& wv, const GatedView& gv,
                                      int64_t add, cudaStream_t s) {
-    const size_t sm = gated_smem(D, gv.h, tv.C);
+    const int warps = gated_warps(D, gv.h);
+    const size_t sm = gated_smem(D, gv.h, warps);
     cudaError_t e = cudaFuncSetAttribute(gated_level_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
@@ -230,12 +236,12 @@ static cudaError_t gated_levels_impl(const TreeView& tv, const WorkView& wv, con
     // an append re-pools a few nodes per unit; a build every node
     const int64_t work = add == 0 ? (int64_t)tv.B * tv.Hkv * ((tv.cap + tv.C - 1) / tv.C)
                                   : (int64_t)tv.B * tv.Hkv * (add / tv.C + 2);
-    int64_t grid = (work + kGatedWarps - 1) / kGatedWarps;
+    int64_t grid = (work + warps - 1) / warps;
     if (grid > nsm) grid = nsm;
     if (grid < 1) grid = 1;
     NvtxRange nv(add == 0 ? "recsa build (gated pooler)" : "recsa append levels (gated pooler)");
     for (int lvl = 1; lvl < tv.n_levels; ++lvl) {
-        gated_level_kernel<T, D><<<(unsigned)grid, kGatedWarps * 32, sm, s>>>(tv, wv, gv, lvl, add);
+        gated_level_kernel<T, D><<<(unsigned)grid, warps * 32, sm, s>>>(tv, wv, gv, lvl, add);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
