@@ -46,8 +46,9 @@ typedef enum {
     RECSA_E_CAPACITY = 3,     /* a length would exceed capacity, or a buffer is too small        */
     RECSA_E_CUDA = 4,         /* a CUDA runtime call or kernel launch failed                      */
     RECSA_E_TIMEOUT = 5,      /* a bounded device wait gave up                                    */
-    RECSA_E_DEVICE = 6        /* device status word: a query or append was out of range, or a    */
-                              /* staging buffer was misaligned                                    */
+    RECSA_E_DEVICE = 6        /* device status word: a query or append was out of range, a       */
+                              /* staging buffer was misaligned, or (bounds-checked build only) an */
+                              /* index failed its range check                                     */
 } recsa_status;
 
 typedef enum { RECSA_F32 = 0, RECSA_BF16 = 1 } recsa_dtype;
