@@ -98,7 +98,7 @@ __device__ __forceinline__ uint32_t swz_off(int half, int row, int chunk, int C)
 // shared-memory layout of the select/attend kernels
 // ----------------------------------------------------------------------------
 struct Smem {
-    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, gs, misc, bars, ring, red, total;
+    size_t qsm, rc4, s, key, nodes, flag, par, mkey, hist, gs, misc, geo, bars, ring, red, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
@@ -125,12 +125,13 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
     L.key = o;   o = align16(o + sizeof(uint32_t) * CH);
     L.nodes = o; o = align16(o + sizeof(int) * CH);
     L.flag = o;  o = align16(o + sizeof(unsigned char) * CH);
-    L.par = o;   o = align16(o + sizeof(int) * 2 * k);   // this level's parents, the next's
+    L.par = o;   o = align16(o + sizeof(int) * 3 * k);   // S^(l) in buffer l mod 3
     const int mk = NA > 0 && NA < 4 * kSelCand ? 4 * kSelCand : NA;
     L.mkey = o;  o = align16(o + sizeof(uint32_t) * mk);
     L.hist = o;  o = align16(o + sizeof(uint32_t) * 1024);   // >= kSelBins / 2, radix 512
     L.gs = o;    o = align16(o + sizeof(uint32_t) * gsw);
     L.misc = o;  o = align16(o + sizeof(int) * 128);
+    L.geo = o;   o = align16(o + sizeof(int) * 4 * kMaxLevels);   // per-level list geometry
     L.bars = o;  o = align16(o + sizeof(uint64_t) * kWarps * 2);
     o = (o + 1023) & ~size_t(1023);   // swizzled slots need 1024-byte alignment
     L.ring = o;
@@ -500,8 +501,9 @@ __device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* m
 //     key.  A bin of more than kSelCand keys (heavy ties) returns false here, in
 //     every CTA alike, and the caller runs the exchange-and-select path instead.
 //  3. Each CTA publishes the (key, position) pairs of its keys in bd and its count
-//     of keys above bd; after a second barrier every CTA gathers all candidates
-//     (then arrives on the cluster barrier that the caller waits on before exit).
+//     of keys above bd; after a second barrier every CTA gathers all candidates.
+//     The caller arrives on the cluster barrier once its remote reads and its
+//     stores of S are done, and waits on it at the end of the level.
 //     The threshold follows from a 256-bin histogram of the candidates' next 8 key
 //     bits and an exact rank of the few candidates in the boundary sub-bin.
 //  4. A selected entry's rank is the count of selected entries in the CTAs before
@@ -591,7 +593,6 @@ __device__ bool cluster_select(const uint32_t* key, int n_loc, int j0, int K, in
     int base_above = 0;
     for (int r = 0; r < crank; ++r) base_above += misc[kMiscGA + r];
     __syncthreads();
-    cluster_arrive();   // remote reads done; the caller waits before exit
 
     // threshold: the sub-bin (next 8 bits) holding the need-th candidate ...
     {
@@ -794,6 +795,7 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int C, in
         asm volatile("prefetch.global.L1 [%0];" ::"l"(rope + (int64_t)(p_q - next_jb) * H + cl * PPL));
     {
         const float4* qcs = reinterpret_cast<const float4*>(rope + (int64_t)(p_q - jb) * H + cl * PPL);
+        const float4* q4 = reinterpret_cast<const float4*>(qsm) + cl * CPL;
 #pragma unroll
         for (int w = 0; w < CPL; ++w) {
             const float4 cs = __ldg(qcs + w);   // (cos v, sin v, cos v+1, sin v+1)
@@ -802,26 +804,35 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int C, in
             const float2 ns = make_float2(-cs.y, -cs.w);
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float2 x1 = *reinterpret_cast<const float2*>(qsm + g * D + cl * PPL + 2 * w);
-                const float2 x2 = *reinterpret_cast<const float2*>(qsm + g * D + H + cl * PPL + 2 * w);
+                const float4 xq = q4[g * (H / 2) + w];   // (low v, low v+1, high v, high v+1)
+                const float2 x1 = make_float2(xq.x, xq.y);
+                const float2 x2 = make_float2(xq.z, xq.w);
                 qlo[g][w] = __ffma2_rn(x2, ns, __fmul2_rn(x1, co));
                 qhi[g][w] = __ffma2_rn(x1, si, __fmul2_rn(x2, co));
             }
         }
     }
+    // swizzled slots: row cb + u*KPW + kg (cb a multiple of KPW*U = 8, so the row's
+    // swizzle phase is u*KPW + kg) keeps the lane's chunk cl/2 at chunk
+    // (cl/2 ^ kg) ^ (u*KPW); the slot always holds C rows, so rows past nch are read
+    // too and their results dropped
+    static_assert(!SW || (KPW == 2 && U == 4), "swizzle phases of the scoring rows");
+    const uint32_t ch0 = (uint32_t)((cl >> 1) ^ kg);
+    const uint32_t rb0 = (uint32_t)kg * 128u + (uint32_t)(cl & 1) * 8u;
     for (int cb = 0; cb < nch; cb += KPW * U) {
         float v[NV];
         // a key past the group reads row 0 (always staged); its value is never stored
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int c = cb + u * KPW + kg;
-            const int cr = c < nch ? c : 0;
+            const int cr = SW ? c : (c < nch ? c : 0);
             float2 kl[CPL], kh[CPL];
             if constexpr (SW) {
                 // the lane's 8 bytes: half of 16-byte chunk cl / 2 of each half row
-                const uint32_t in = (uint32_t)(cl & 1) * 8u;
-                PairLoad<T, PPL>::get(blk + swz_off(0, cr, cl >> 1, C) + in, kl);
-                PairLoad<T, PPL>::get(blk + swz_off(1, cr, cl >> 1, C) + in, kh);
+                const unsigned char* row =
+                    blk + (uint32_t)cb * 128u + rb0 + (uint32_t)(u * KPW) * 128u + ((ch0 ^ (uint32_t)(u * KPW)) << 4);
+                PairLoad<T, PPL>::get(row, kl);
+                PairLoad<T, PPL>::get(row + C * 128, kh);
             } else {
                 const unsigned char* row = blk + cr * kRow;
                 PairLoad<T, PPL>::get(row + off, kl);
@@ -890,20 +901,52 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int C, in
     }
 }
 
-// Unrotated query heads of one KV head (fp32) and the C child rotations R(c) into
+// Unrotated query heads of one KV head (fp32, as couples: float4 (low v, low v+1,
+// high v, high v+1) of pairs v, v+1 at [g][v/2]) and the C child rotations R(c) into
 // shared memory.  R(c) is stored per pair couple (v, v+1) as (cos v, cos v+1,
 // sin v, sin v+1); couple w of the lane that owns couples [CPL*l, CPL*l + CPL)
 // sits at c * (D/4) + w * LPK + l, so the LPK lanes of one key read consecutive
-// 16-byte words.
+// 16-byte words.  Every global load of the thread is issued before its first
+// shared-memory store, so the loads overlap instead of waiting one by one.
 template <typename T, int D, int G>
 __device__ __forceinline__ void stage_query(const T* qrow, const float2* rope, int C, float* qsm,
                                             float4* rc4) {
     using S = Shape<T, D>;
-    for (int i = threadIdx.x; i < G * D; i += kThreads) qsm[i] = (float)qrow[i];
-    for (int i = threadIdx.x; i < C * (D / 4); i += kThreads) {
-        const int c = i / (D / 4), f = i % (D / 4);
-        const float2 a = rope[2 * i], bb = rope[2 * i + 1];
-        rc4[c * (D / 4) + (f % S::CPL) * S::LPK + f / S::CPL] = make_float4(a.x, bb.x, a.y, bb.y);
+    constexpr int QN = (G * D + kThreads - 1) / kThreads;
+    constexpr int RN = (RECSA_MAX_C * (D / 4) + kThreads - 1) / kThreads;
+    const int nr = C * (D / 4);
+    float qv[QN];
+    float2 ra[RN], rb[RN];
+#pragma unroll
+    for (int u = 0; u < QN; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        qv[u] = i < G * D ? (float)qrow[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < RN; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        ra[u] = rb[u] = make_float2(0.f, 0.f);
+        if (i < nr) {
+            ra[u] = rope[2 * i];
+            rb[u] = rope[2 * i + 1];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < QN; ++u) {
+        // dim d of head g at couple d/2 (low half) or (d-H)/2 (high half) of head g:
+        // float4 (low v, low v+1, high v, high v+1)
+        const int i = threadIdx.x + u * kThreads;
+        const int g = i / D, d = i % D, hi = d >= D / 2, dd = hi ? d - D / 2 : d;
+        if (i < G * D) qsm[(g * (D / 4) + dd / 2) * 4 + 2 * hi + (dd & 1)] = qv[u];
+    }
+#pragma unroll
+    for (int u = 0; u < RN; ++u) {
+        const int i = threadIdx.x + u * kThreads;
+        if (i < nr) {
+            const int c = i / (D / 4), f = i % (D / 4);
+            rc4[c * (D / 4) + (f % S::CPL) * S::LPK + f / S::CPL] =
+                make_float4(ra[u].x, rb[u].x, ra[u].y, rb[u].y);
+        }
     }
 }
 
@@ -1176,16 +1219,36 @@ __device__ void combine_unit(const float* P, int lstar, int SPL, int NS0, int NL
     float* vals = ll + G * ns;   // [ns][E] staged values
     auto slot_of = [&](int i) { return i < nls ? i : NL * SPL + (i - nls); };
     const int cap = (nbuf - 3 * G * ns) / ns;   // output elements staged per round
-    // (m, l) of every slot and head, and the first round of values, in one batch
+    // (m, l) of every slot and head, then the first round of values.  The code runs
+    // once per launch (its instructions are fetched cold), so it stays short: no
+    // division per element, and KB loads of a thread in flight before their stores.
+    constexpr int KB = 8;
     const int E0 = min(cap, e1 - e0);
-    for (int x = threadIdx.x; x < ns * G + ns * E0; x += kThreads) {
-        if (x < ns * G) {
-            const int i = x / G, g = x % G;
-            const float* rec = P + (slot_of(i) * G + g) * (D + 2);
-            mm[g * ns + i] = __ldcg(rec + D);
-            ll[g * ns + i] = __ldcg(rec + D + 1);
-        } else {
-            const int y = x - ns * G;
+    for (int x = threadIdx.x; x < ns * G; x += kThreads) {
+        const int i = x / G, g = x % G;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(P + (slot_of(i) * G + g) * (D + 2) + D));
+        mm[g * ns + i] = ml.x;
+        ll[g * ns + i] = ml.y;
+    }
+    // thread -> column e0 + c of slots i0, i0 + di, ... (when E0 divides kThreads)
+    const bool cols = kThreads % E0 == 0;
+    const int c = cols ? threadIdx.x % E0 : 0, i0 = cols ? threadIdx.x / E0 : 0;
+    const int di = cols ? kThreads / E0 : 1;
+    const float* colp = P + ((e0 + c) / D) * (D + 2) + (e0 + c) % D;
+    if (cols) {
+        for (int ib = i0; ib < ns; ib += KB * di) {
+            float v[KB];
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const int i = ib + u * di;
+                v[u] = i < ns ? __ldcg(colp + slot_of(i) * G * (D + 2)) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < KB; ++u)
+                if (ib + u * di < ns) vals[(ib + u * di) * E0 + c] = v[u];
+        }
+    } else {
+        for (int y = threadIdx.x; y < ns * E0; y += kThreads) {
             const int i = y / E0, e = e0 + y % E0;
             vals[y] = __ldcg(P + (slot_of(i) * G + e / D) * (D + 2) + e % D);
         }
@@ -1284,10 +1347,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t* key = reinterpret_cast<uint32_t*>(smem + SL.key);
     int* nodes = reinterpret_cast<int*>(smem + SL.nodes);
     unsigned char* flag = smem + SL.flag;
-    // par: S^(level+1), the parents of this level's list (entries this CTA needs);
-    // par_next: S^(level), filled by the cluster's CTAs as they select
-    int* par = reinterpret_cast<int*>(smem + SL.par);
-    int* par_next = par + k;
+    // S^(l), as far as this CTA needs it, in buffer l mod 3: at a level the CTA reads
+    // its parents S^(level+1) while the cluster's CTAs store S^(level) into the next
+    // buffer, and a CTA that runs one level ahead stores S^(level-1) into the third
+    int* pbuf = reinterpret_cast<int*>(smem + SL.par);
     uint32_t* mkey = reinterpret_cast<uint32_t*>(smem + SL.mkey);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + SL.hist);
     uint32_t* gs = reinterpret_cast<uint32_t*>(smem + SL.gs);
@@ -1358,11 +1421,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     // written (only L2 prefetch hints go out above): the kernel just before may be
     // the caller's own, writing q.
     pdl_wait();
-    stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
     const int64_t len = wv.lens[b];
+    stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
     const int64_t t = (qv.mode == 0) ? len - 1 : qv.pos0 + (gq - b * qv.n_per_b);
     const bool valid = t >= 0 && t < len;
     const int lstar = valid ? first_scored_level(t, C, lgC, k) : 0;
+    // the list geometry of every level, one thread per level (each a chain of
+    // dependent integer steps): |A^(l)|, the entries per CTA, and the parents per
+    // CTA of the level below
+    int* geo = reinterpret_cast<int*>(smem + SL.geo);
+    if (valid && threadIdx.x <= lstar) {
+        const int l = threadIdx.x;
+        const int nA_l = list_size(t, lstar, l, C, lgC, k);
+        const int npar_l = cdiv(nA_l + C - 1, C, lgC);
+        geo[4 * l] = nA_l;
+        geo[4 * l + 1] = ((npar_l + nsplit - 1) / nsplit) * C;
+        if (l >= 1) {
+            const int nA_m = list_size(t, lstar, l - 1, C, lgC, k);
+            geo[4 * l + 2] = (cdiv(nA_m + C - 1, C, lgC) + nsplit - 1) / nsplit;
+        }
+    }
     int32_t* cnt_ws = wv.cnt + (int64_t)unit * (NL + 1);
     int32_t* cnt_usr = qv.cnt_out ? qv.cnt_out + ((int64_t)gq * tv.Hkv + kvh) * (NL + 1) : nullptr;
     float* part = wv.part + (int64_t)unit * wv.NSLOT * G * (D + 2);
@@ -1399,33 +1477,32 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (level > lstar) continue;   // not scored: recorded after the pass
         if (qv.phase == 2 && !L0) continue;   // levels >= 1 were done by the phase-1 launch
         if (qv.phase == 1 && L0) break;       // level 0 and the merge: the phase-2 launch
-        if (level < lstar) {
-            // the parent list S^(level+1): every CTA of the cluster has stored the
-            // entries this CTA needs into its par_next; after the barrier they are in
-            // place, and every CTA is past the level above
-            cluster.sync();
-            int* tmp = par;
-            par = par_next;
-            par_next = tmp;
-        }
+        // Below the first scored level no barrier is needed here: every CTA of the
+        // cluster stored its part of S^(level+1) into the other CTAs' buffers, and
+        // zeroed its slice of the selection's global histogram, before the cluster
+        // arrive that the level above waited on at its end.
+        const int* par = pbuf + ((level + 1) % 3) * k;
+        int* par_next = pbuf + (level % 3) * k;
+        const bool first = level == lstar;
         if (!L0) {
-            // the selection's histograms and published counts start at zero in every
-            // CTA of the cluster before any CTA adds into them (waited on after the
-            // scores).  Done first at a level, so the release has no other stores of
-            // this CTA to wait for.
+            // this CTA's own histogram and counters (peers read the counters only
+            // after the selection's second barrier)
             for (int i = threadIdx.x; i < kSelBins / 2; i += kThreads) hist[i] = 0u;
-            for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
             if (threadIdx.x == 0) misc[kMiscPubC] = misc[kMiscPubA] = 0;
-            __syncthreads();
-            cluster_arrive();
+            if (first) {
+                // the global histogram's slices start at zero in every CTA before any
+                // CTA adds into them (waited on after the scores)
+                for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
+                __syncthreads();
+                cluster_arrive();
+            }
         } else {
             pdl_launch_dependents();   // the next kernel may start launching
         }
-        const int nA = list_size(t, lstar, level, C, lgC, k);
+        const int nA = geo[4 * level];
         // phase 2 reads level 0 from the staging copy, where entry j is row j
         const bool identity = level == lstar || qv.phase == 2;
-        const int npar_all = cdiv(nA + C - 1, C, lgC);
-        const int chunk = ((npar_all + nsplit - 1) / nsplit) * C;
+        const int chunk = geo[4 * level + 1];
         const int j0 = split * chunk;
         const int j1 = min(nA, j0 + chunk);
         const T *kbase, *vbase;
@@ -1457,12 +1534,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                : qv.sel_out + (((int64_t)gq * tv.Hkv + kvh) * NL + (level - 1)) * k;
         float* outp = part + (int64_t)((L0 ? NL * wv.SPL : (level - 1) * wv.SPL) + split) * G * (D + 2);
         // parents per CTA at the next level: parent rank r goes to CTA r / ppc_next
-        int ppc_next = 1;
-        if (!L0) {
-            const int nA_next = list_size(t, lstar, level - 1, C, lgC, k);
-            const int npar_next = cdiv(nA_next + C - 1, C, lgC);
-            ppc_next = (npar_next + nsplit - 1) / nsplit;
-        }
+        const int ppc_next = L0 ? 1 : geo[4 * level + 2];
         if (!L0 && nA <= k) {
             // everything selected, no summaries (not reachable below the first scored
             // level when k, C >= 2; kept for completeness)
@@ -1478,8 +1550,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
             write_empty_partial(outp, G, D);
+            if (first) cluster_wait();   // the arrive at the level's start
+            for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
             __syncthreads();
-            cluster_wait();   // matches the arrive at the level's start
+            cluster_arrive();   // S^(level) stored, the slice zeroed for the level below
+            cluster_wait();
             continue;
         }
 
@@ -1550,7 +1625,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         if (!L0) {
             const int M = nA - 1;
-            cluster_wait();   // every CTA's zeroed histograms (and keys) are in place
+            if (first) cluster_wait();   // every CTA's zeroed histogram slice is in place
             // 2. exact top-(k-1) over all M keys; this CTA writes S for its entries
             auto mark = [&](int i, int r) {
                 if (!in_bounds(r >= 0 && r < K1 && i >= j0 && i < j0 + n_sc &&
@@ -1567,8 +1642,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint2* pub = reinterpret_cast<uint2*>(mkey);
                 done = cluster_select(key, n_sc, j0, K1, csize, crank, gsw, hist, gs, pub,
                                       pub + kSelCand, misc, mark);
-            } else {
-                cluster_arrive();
             }
             if (!done) {
                 // heavy ties: every CTA's keys in list order (list position = merged
@@ -1580,7 +1653,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll 4
                     for (int i = threadIdx.x; i < hi - lo; i += kThreads) mkey[lo + i] = rk[i];
                 }
-                cluster_arrive();   // remote reads done; matched by cluster_wait() below
                 __syncthreads();
                 select_topk(mkey, M, K1, hist, misc, j0, j0 + n_sc, mark);
             }
@@ -1590,7 +1662,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (sel_usr) sel_usr[K1] = (int)cur;
                 cluster.map_shared_rank(par_next, K1 / ppc_next)[K1] = (int)cur;
             }
+            // every remote read of this level is done (the other CTAs' keys, candidates,
+            // counts and histogram slices) and every store of S^(level) into the other
+            // CTAs has been issued; the slice is zeroed for the level below.  The
+            // release publishes both; the level's end waits for every CTA.
+            for (int i = threadIdx.x; i < gsw; i += kThreads) gs[i] = 0u;
             __syncthreads();
+            cluster_arrive();
             // No L2 prefetch of the kept nodes' children here: bulk prefetches queue in
             // the same TMA unit as the rings' copies, and delayed this level's value
             // blocks and the next level's first blocks by more than they saved.
@@ -1640,7 +1718,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // red (the ring) is read: the next level's tensor copies may overwrite it
         __syncthreads();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (!L0) cluster_wait();   // matches the arrive after this CTA's remote reads
+        if (!L0) cluster_wait();   // every CTA's arrive after its selection
     }
 
     if (split == 0 && qv.phase != 2) {
