@@ -149,8 +149,10 @@ __host__ __device__ inline Smem smem_layout(int G, int D, int CH, int k, int C, 
 enum { kMiscDigit = 0, kMiscAbove = 1, kMiscCount = 2, kMiscScan = 4 /* kWarps+1 */,
        kMiscFloat = 16 /* 2*G floats */, kMiscLast = 40, kMiscN = 41,
        // cluster selection: published counts, gathered counts (one per CTA), scalars
-       kMiscPubC = 48, kMiscPubA = 49, kMiscSB = 50, kMiscSBAbove = 51, kMiscMemN = 52,
-       kMiscTk = 53, kMiscTj = 54, kMiscGC = 64 /* 16 */, kMiscGA = 80 /* 16 */,
+       kMiscPubC = 48, kMiscPubA = 49, kMiscTk = 53, kMiscTj = 54, kMiscGC = 64 /* 16 */,
+       kMiscGA = 80 /* 16 */,
+       kMiscWA = 104 /* kWarps: keys above the boundary bin per slice */,
+       kMiscBase = 112 /* kWarps: first rank of each slice */,
        kMiscFailed = 100 /* a bounded wait of this CTA gave up */ };
 
 // Split cluster barrier: arrive (release) and, later, wait (acquire); every thread
@@ -497,18 +499,21 @@ __device__ void select_topk(uint32_t* mkey, int M, int K, uint32_t* hist, int* m
 //     are spread over the CTAs (gsw words each, zeroed by the caller before a
 //     cluster arrive that the caller's wait completed): distributed shared memory
 //     atomics.  A cluster barrier follows.
-//  2. Every CTA reads the global histogram and finds the bin bd holding the K-th
-//     key.  A bin of more than kSelCand keys (heavy ties) returns false here, in
-//     every CTA alike, and the caller runs the exchange-and-select path instead.
-//  3. Each CTA publishes the (key, position) pairs of its keys in bd and its count
-//     of keys above bd; after a second barrier every CTA gathers all candidates.
-//     The caller arrives on the cluster barrier once its remote reads and its
-//     stores of S are done, and waits on it at the end of the level.
-//     The threshold follows from a 256-bin histogram of the candidates' next 8 key
-//     bits and an exact rank of the few candidates in the boundary sub-bin.
-//  4. A selected entry's rank is the count of selected entries in the CTAs before
-//     this one (their counts above bd plus their selected candidates) plus its
-//     rank within this CTA.
+//  2. Every CTA reads the global histogram (one 16-byte remote load per thread) and
+//     finds the bin bd holding the K-th key with warp scans.  A bin of more than
+//     kSelCand keys (heavy ties) returns false here, in every CTA alike, and the
+//     caller runs the exchange-and-select path instead.
+//  3. Each warp takes a slice of the CTA's keys in list order, publishes the (key,
+//     position) pairs of its keys in bd and counts its keys above bd; after a
+//     second barrier every CTA gathers all candidates and their counts.  The
+//     caller arrives on the cluster barrier once its remote reads and its stores
+//     of S are done, and waits on it at the end of the level.
+//  4. Warp 0 finds the threshold from a 256-bin histogram of the candidates' next 8
+//     key bits and an exact rank of the few candidates in the boundary sub-bin,
+//     and the rank at which each slice starts: the selected entries of the CTAs
+//     before this one (their counts above bd plus their selected candidates) and
+//     of the slices before it.
+//  5. Each warp ranks its slice's selected entries with ballots.
 // ----------------------------------------------------------------------------
 template <typename Fn>
 __device__ bool cluster_select(const uint32_t* key, int n_loc, int j0, int K, int csize, int crank,
@@ -540,49 +545,83 @@ __device__ bool cluster_select(const uint32_t* key, int n_loc, int j0, int K, in
     cluster.sync();
 
     // 2. the global histogram: thread t owns bins kSelBins-1-BPT*t-u, the words
-    //    from W-4-4t (bin b: word b/2, high half when b is odd)
+    //    from W-4-4t (bin b: word b/2, high half when b is odd).  Keys above a
+    //    thread's bins: a warp scan plus the totals of the warps before it.
     {
         const int w0 = W - 4 - 4 * tid;
         const uint4 w = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(gs, w0 / gsw) + w0 % gsw);
         const uint32_t ws[4] = {w.w, w.z, w.y, w.x};
         uint32_t cnt8[BPT];
+        int tot = 0;
 #pragma unroll
-        for (int u = 0; u < BPT; ++u) cnt8[u] = (ws[u >> 1] >> (16 * (1 - (u & 1)))) & 0xFFFFu;
-        find_boundary_bin<BPT>(cnt8, K, misc);
+        for (int u = 0; u < BPT; ++u) {
+            cnt8[u] = (ws[u >> 1] >> (16 * (1 - (u & 1)))) & 0xFFFFu;
+            tot += (int)cnt8[u];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) misc[kMiscScan + warp] = incl;
+        __syncthreads();
+        int run = incl - tot;
+        for (int ww = 0; ww < warp; ++ww) run += misc[kMiscScan + ww];
+        if (run < K && K <= run + tot) {
+#pragma unroll
+            for (int u = 0; u < BPT; ++u) {
+                if (run < K && K <= run + (int)cnt8[u]) {
+                    misc[kMiscDigit] = kSelBins - 1 - BPT * tid - u;
+                    misc[kMiscAbove] = run;
+                    misc[kMiscCount] = (int)cnt8[u];
+                }
+                run += (int)cnt8[u];
+            }
+        }
+        __syncthreads();
     }
     const uint32_t bd = (uint32_t)misc[kMiscDigit];
     const int cnt = misc[kMiscCount];
     if (cnt > kSelCand) return false;
     const int need = K - misc[kMiscAbove];   // 1..cnt
+    const unsigned lt = (1u << lane) - 1u;
 
-    // 3. this CTA's candidates and its count above bd, for the other CTAs
-    int my_above = 0;
-    for (int i0 = 0; i0 < n_loc; i0 += kThreads) {
-        const int i = i0 + tid;
-        const uint32_t kk = i < n_loc ? key[i] : 0u;
-        const uint32_t dig = kk >> SH;
-        const bool in = i < n_loc && dig == bd;
-        my_above += (i < n_loc && dig > bd) ? 1 : 0;
-        const unsigned bal = __ballot_sync(kFull, in);
-        if (bal) {
-            int base = 0;
-            if (lane == 0) base = atomicAdd(&misc[kMiscPubC], __popc(bal));
-            base = __shfl_sync(kFull, base, 0);
-            if (in) pub[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(kk, (uint32_t)(j0 + i));
+    // 3. this CTA's candidates and its count above bd, for the other CTAs; each warp
+    //    takes a slice of the keys in list order and counts its keys above bd
+    const int per = (((n_loc + kWarps - 1) / kWarps) + 31) & ~31;
+    const int s0 = warp * per, s1 = min(n_loc, s0 + per);
+    {
+        int wab = 0;
+        for (int i = s0 + lane; i - lane < s1; i += 32) {
+            const bool v = i < s1;
+            const uint32_t kk = v ? key[i] : 0u;
+            const uint32_t dig = kk >> SH;
+            const bool in = v && dig == bd;
+            wab += __popc(__ballot_sync(kFull, v && dig > bd));
+            const unsigned bal = __ballot_sync(kFull, in);
+            if (bal) {
+                int base = 0;
+                if (lane == 0) base = atomicAdd(&misc[kMiscPubC], __popc(bal));
+                base = __shfl_sync(kFull, base, 0);
+                if (in) pub[base + __popc(bal & lt)] = make_uint2(kk, (uint32_t)(j0 + i));
+            }
+        }
+        if (lane == 0) {
+            misc[kMiscWA + warp] = wab;
+            if (wab) atomicAdd(&misc[kMiscPubA], wab);
         }
     }
-    my_above = (int)__reduce_add_sync(kFull, (unsigned)my_above);
-    if (lane == 0 && my_above) atomicAdd(&misc[kMiscPubA], my_above);
     cluster.sync();
     if (tid < csize) {
         const int* rm = cluster.map_shared_rank(misc, tid);
         misc[kMiscGC + tid] = rm[kMiscPubC];
         misc[kMiscGA + tid] = rm[kMiscPubA];
     }
-    uint32_t* sub = lh;   // free since step 1: sub-bin counts, then the member list
+    uint32_t* sub = lh;   // free since step 1: sub-bin counts, then the members
     sub[tid] = 0u;
-    if (tid == 0) misc[kMiscMemN] = 0;
     __syncthreads();
+    // 4. every CTA's candidates, with a histogram of their next 8 key bits
     for (int idx = tid; idx < cnt; idx += kThreads) {
         int r = 0, off = 0;
         while (r < csize - 1 && idx >= off + misc[kMiscGC + r]) off += misc[kMiscGC + r++];
@@ -590,73 +629,106 @@ __device__ bool cluster_select(const uint32_t* key, int n_loc, int j0, int K, in
         all[idx] = c;
         atomicAdd(&sub[(c.x >> (SH - 8)) & 255u], 1u);
     }
-    int base_above = 0;
-    for (int r = 0; r < crank; ++r) base_above += misc[kMiscGA + r];
     __syncthreads();
 
-    // threshold: the sub-bin (next 8 bits) holding the need-th candidate ...
-    {
-        const int c = (int)sub[255 - tid];
-        int tot;
-        const int ex = block_excl_scan(c, misc + kMiscScan, tot);
-        if (ex < need && need <= ex + c) {
-            misc[kMiscSB] = 255 - tid;
-            misc[kMiscSBAbove] = ex;
+    // 5. warp 0: the threshold (the sub-bin holding the need-th candidate, then an
+    //    exact rank of its members) and the rank at which each warp's slice starts
+    // (rolled loops over the candidates in shared memory: this code runs once per
+    // level in one warp, and its instructions often arrive cold)
+    if (warp == 0) {
+        // lane l holds sub-bins [8l, 8l + 8); higher lanes hold higher keys
+        const uint4 h0 = *reinterpret_cast<const uint4*>(sub + 8 * lane);
+        const uint4 h1 = *reinterpret_cast<const uint4*>(sub + 8 * lane + 4);
+        const uint32_t h8[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        uint32_t t8 = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) t8 += h8[u];
+        uint32_t suf = t8;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(kFull, suf, o);
+            if (lane + o < 32) suf += y;
         }
-        __syncthreads();
-    }
-    const uint32_t sb = (uint32_t)misc[kMiscSB];
-    const int need2 = need - misc[kMiscSBAbove];
-    // ... and the exact rank of each candidate in that sub-bin among the others there
-    for (int i0 = 0; i0 < cnt; i0 += kThreads) {
-        const int idx = i0 + tid;
-        const bool in = idx < cnt && ((all[idx].x >> (SH - 8)) & 255u) == sb;
-        const unsigned bal = __ballot_sync(kFull, in);
-        if (bal) {
-            int base = 0;
-            if (lane == 0) base = atomicAdd(&misc[kMiscMemN], __popc(bal));
-            base = __shfl_sync(kFull, base, 0);
-            if (in) sub[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)idx;
+        uint32_t srun = suf - t8;
+        const unsigned hit = __ballot_sync(kFull, srun < (uint32_t)need && (uint32_t)need <= suf);
+        const int src = hit ? __ffs(hit) - 1 : 0;
+        int sbl = 0, sba = 0;
+        bool found = false;
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+            if (!found) {
+                if (srun + h8[u] >= (uint32_t)need) { found = true; sbl = 8 * lane + u; sba = (int)srun; }
+                else srun += h8[u];
+            }
         }
-    }
-    __syncthreads();
-    const int nm = misc[kMiscMemN];
-    for (int mi = warp; mi < nm; mi += kWarps) {
-        const uint2 me = all[sub[mi]];
-        int gt = 0;
-        for (int o = lane; o < nm; o += 32) {
-            const uint2 x = all[sub[o]];
-            gt += (x.x > me.x || (x.x == me.x && x.y < me.y)) ? 1 : 0;
+        const uint32_t sb = (uint32_t)__shfl_sync(kFull, sbl, src);
+        const int need2 = need - __shfl_sync(kFull, sba, src);
+        __syncwarp();   // the sub-bin counts are read: their words take the members
+        uint2* memb = reinterpret_cast<uint2*>(sub);
+        int nm = 0;
+#pragma unroll 1
+        for (int i0 = 0; i0 < cnt; i0 += 32) {
+            const int idx = i0 + lane;
+            const uint2 c = idx < cnt ? all[idx] : make_uint2(0u, 0u);
+            const bool in = idx < cnt && ((c.x >> (SH - 8)) & 255u) == sb;
+            const unsigned bal = __ballot_sync(kFull, in);
+            if (in) memb[nm + __popc(bal & lt)] = c;
+            nm += __popc(bal);
         }
-        gt = (int)__reduce_add_sync(kFull, (unsigned)gt);
-        if (lane == 0 && gt == need2 - 1) {
-            misc[kMiscTk] = (int)me.x;
-            misc[kMiscTj] = (int)me.y;
+        __syncwarp();
+        uint32_t Tk = 0u, Tj = 0u;
+#pragma unroll 1
+        for (int mi = lane; mi - lane < nm; mi += 32) {
+            const uint2 me = mi < nm ? memb[mi] : make_uint2(0u, 0u);
+            int gt = 0;
+            for (int o = 0; o < nm; ++o) {
+                const uint2 xo = memb[o];
+                gt += (xo.x > me.x || (xo.x == me.x && xo.y < me.y)) ? 1 : 0;
+            }
+            const unsigned hb = __ballot_sync(kFull, mi < nm && gt == need2 - 1);
+            if (hb) {
+                const int sl = __ffs(hb) - 1;
+                Tk = __shfl_sync(kFull, me.x, sl);
+                Tj = __shfl_sync(kFull, me.y, sl);
+            }
+        }
+        // selected candidates before this CTA, and in each slice of this CTA (added
+        // into kMiscWA, which holds each slice's keys above bd)
+        int before = 0;
+#pragma unroll 1
+        for (int idx = lane; idx < cnt; idx += 32) {
+            const uint2 c = all[idx];
+            const bool sel = c.x > Tk || (c.x == Tk && c.y <= Tj);
+            const int li = (int)c.y - j0;
+            before += (sel && li < 0) ? 1 : 0;
+            if (sel && li >= 0 && li < n_loc) atomicAdd(&misc[kMiscWA + li / per], 1);
+        }
+        before = (int)__reduce_add_sync(kFull, (unsigned)before);
+        const int above_before =
+            (int)__reduce_add_sync(kFull, (unsigned)(lane < crank ? misc[kMiscGA + lane] : 0));
+        __syncwarp();
+        if (lane == 0) {
+            int base = above_before + before;
+            for (int ww = 0; ww < kWarps; ++ww) {
+                misc[kMiscBase + ww] = base;
+                base += misc[kMiscWA + ww];
+            }
+            misc[kMiscTk] = (int)Tk;
+            misc[kMiscTj] = (int)Tj;
         }
     }
     __syncthreads();
     const uint32_t T = (uint32_t)misc[kMiscTk], jT = (uint32_t)misc[kMiscTj];
 
-    // 4. ranks: selected candidates of the CTAs before this one, then this CTA's
-    int sc = 0;
-    for (int idx = tid; idx < cnt; idx += kThreads) {
-        const uint2 c = all[idx];
-        sc += (c.y < (uint32_t)j0 && (c.x > T || (c.x == T && c.y <= jT))) ? 1 : 0;
-    }
-    int sel_before;
-    block_excl_scan(sc, misc + kMiscScan, sel_before);
-    const int ipt = (n_loc + kThreads - 1) / kThreads;
-    const int i0 = tid * ipt, i1 = min(n_loc, i0 + ipt);
-    int cs = 0;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t kk = key[i];
-        cs += (kk > T || (kk == T && (uint32_t)(j0 + i) <= jT)) ? 1 : 0;
-    }
-    int tot;
-    int r = base_above + sel_before + block_excl_scan(cs, misc + kMiscScan, tot);
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t kk = key[i];
-        if (kk > T || (kk == T && (uint32_t)(j0 + i) <= jT)) mark(j0 + i, r++);
+    // 6. this warp's selected entries, ranked in list order
+    int r = misc[kMiscBase + warp];
+    for (int i = s0 + lane; i - lane < s1; i += 32) {
+        const bool v = i < s1;
+        const uint32_t kk = v ? key[i] : 0u;
+        const bool sel = v && (kk > T || (kk == T && (uint32_t)(j0 + i) <= jT));
+        const unsigned bal = __ballot_sync(kFull, sel);
+        if (sel) mark(j0 + i, r + __popc(bal & lt));
+        r += __popc(bal);
     }
     return true;
 }
