@@ -845,11 +845,11 @@ __device__ __forceinline__ const unsigned char* ring_wait(const WarpRing& R, int
 // products are combined by a reduce-scatter over the LPK lanes.
 // ----------------------------------------------------------------------------
 template <typename T, int D, int G, bool WITH_KEY, bool SW>
-__device__ __forceinline__ void score_parent(const unsigned char* blk, int C, int jb, int next_jb,
-                                             int j0, int nch, int64_t first, const float2* rope,
-                                             int p_q,
-                                             const float4* rc4, const float* qsm, float scale,
-                                             float* s, uint32_t* key, int* nodes, int CH) {
+__device__ __forceinline__ void score_parent(const unsigned char* blk, int C, int jb,
+                                             const float4 (&qcs)[Shape<T, D>::CPL], int j0, int nch,
+                                             int64_t first, const float4* rc4, const float* qsm,
+                                             float scale, float* s, uint32_t* key, int* nodes,
+                                             int CH) {
     using S = Shape<T, D>;
     constexpr int LPK = S::LPK, PPL = S::PPL, CPL = S::CPL, KPW = S::KPW, H = D / 2;
     constexpr int kRow = D * (int)sizeof(T);
@@ -861,16 +861,14 @@ __device__ __forceinline__ void score_parent(const unsigned char* blk, int C, in
     const int lane = threadIdx.x & 31;
     const int cl = lane % LPK, kg = lane / LPK;
     const int off = cl * PPL * (int)sizeof(T);   // byte offset of the lane's pairs in a half
-    // the query heads rotated by R(p_q - jb), the lane's couples only
+    // the query heads rotated by R(p_q - jb), the lane's couples only; qcs holds the
+    // lane's couples of that rotation, loaded by the caller a group ahead
     float2 qlo[G][CPL], qhi[G][CPL];
-    if (next_jb >= 0)   // the warp's next group: its rope row into L1 while this one runs
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(rope + (int64_t)(p_q - next_jb) * H + cl * PPL));
     {
-        const float4* qcs = reinterpret_cast<const float4*>(rope + (int64_t)(p_q - jb) * H + cl * PPL);
         const float4* q4 = reinterpret_cast<const float4*>(qsm) + cl * CPL;
 #pragma unroll
         for (int w = 0; w < CPL; ++w) {
-            const float4 cs = __ldg(qcs + w);   // (cos v, sin v, cos v+1, sin v+1)
+            const float4 cs = qcs[w];   // (cos v, sin v, cos v+1, sin v+1)
             const float2 co = make_float2(cs.x, cs.z);
             const float2 si = make_float2(cs.y, cs.w);
             const float2 ns = make_float2(-cs.y, -cs.w);
@@ -1679,15 +1677,28 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             __syncwarp();
         } else {
+            // the rotation R(p_q - jb) of each group, the lane's couples, loaded one
+            // group ahead into registers
+            constexpr int CPL = Shape<T, D>::CPL;
+            const int qoff = (lane % Shape<T, D>::LPK) * Shape<T, D>::PPL;
+            float4 qcs[CPL];
+            auto load_qcs = [&](int jb_, float4 (&o)[CPL]) {
+                const float4* r = reinterpret_cast<const float4*>(wv.rope + (int64_t)(p_q - jb_) * (D / 2) + qoff);
+#pragma unroll
+                for (int w = 0; w < CPL; ++w) o[w] = __ldg(r + w);
+            };
+            if (nw > 0) load_qcs(j0 + warp * C, qcs);
             for (int i = 0; i < nw; ++i) {
                 const unsigned char* blk = ring_wait(R, qbase + i);
                 const int jb = j0 + (warp + kWarps * i) * C;
                 const int nch = min(C, j0 + n_sc - jb);
-                const int next_jb = (i + 1 < nw) ? jb + kWarps * C : -1;
+                float4 qn[CPL];
+                if (i + 1 < nw) load_qcs(jb + kWarps * C, qn);
                 if (nch > 0)
-                    score_parent<T, D, G, true, SW>(blk, C, jb, next_jb, j0, nch, group_first(jb),
-                                                    wv.rope, p_q, rc4, qsm, tv.scale, s, key,
-                                                    nodes, CH);
+                    score_parent<T, D, G, true, SW>(blk, C, jb, qcs, j0, nch, group_first(jb), rc4,
+                                                    qsm, tv.scale, s, key, nodes, CH);
+#pragma unroll
+                for (int w = 0; w < CPL; ++w) qcs[w] = qn[w];
                 __syncwarp();
                 if (lane == 0 && i + nsw < nk + nw) issue(i + nsw);
             }
