@@ -75,44 +75,61 @@ __device__ void gated_pool_node(const T* sk, const T* sv, int64_t rs, int m, con
     const double dm = (double)m;
 #pragma unroll
     for (int e = 0; e < N; ++e) mu[e] /= dm;
-    // 2. each child's projection w . (x_c - mu) and the squared deviations
+    // 2. each child's projection w . (x_c - mu) and the squared deviations, four
+    //    children at a time so that their warp reductions overlap
     double ss = 0.0;
-    for (int c = 0; c < m; ++c) {
-        double x[N];
-        load_dims<T, N>(sk + c * rs, off, x);
-        double dw = 0.0;
+    for (int c0 = 0; c0 < m; c0 += 4) {
+        double dw[4];
 #pragma unroll
-        for (int e = 0; e < N; ++e) {
-            const double dx = x[e] - mu[e];
-            dw = fma(dx, w[off + e], dw);
-            ss = fma(dx, dx, ss);
+        for (int u = 0; u < 4; ++u) {
+            dw[u] = 0.0;
+            if (c0 + u < m) {
+                double x[N];
+                load_dims<T, N>(sk + (c0 + u) * rs, off, x);
+#pragma unroll
+                for (int e = 0; e < N; ++e) {
+                    const double dx = x[e] - mu[e];
+                    dw[u] = fma(dx, w[off + e], dw[u]);
+                    ss = fma(dx, dx, ss);
+                }
+            }
         }
-        dw = warp_sum_f64(dw);
-        if (lane == 0) al[c] = dw;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dw[u] += __shfl_xor_sync(kFull, dw[u], o);
+        if (lane == 0)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c0 + u < m) al[c0 + u] = dw[u];
     }
     ss = warp_sum_f64(ss);
     const double sigma = sqrt(ss / (dm * (double)D) + 1e-6);
     __syncwarp();
-    // 3. softmax over the children of tau * projection / sigma: lane c < m forms
-    //    exp(logit_c - max) once; the sum is taken in child order
-    double mx = -INFINITY;
-    for (int c = 0; c < m; ++c) mx = fmax(mx, gv.tau * al[c] / sigma);
+    // 3. softmax over the children of (tau / sigma) * projection: lane c < m (m <= 32)
+    //    forms its child's logit, the maximum is a warp reduction, and
+    //    exp(logit_c - max) is formed once; the sum is taken in child order
+    const double ts = gv.tau / sigma;
+    const double lg = lane < m ? ts * al[lane] : -INFINITY;
+    const double mx = warp_max_f64(lg);
     __syncwarp();
-    for (int c = lane; c < m; c += 32) al[c] = exp(gv.tau * al[c] / sigma - mx);
+    if (lane < m) al[lane] = exp(lg - mx);
     __syncwarp();
     double sum = 0.0;
     for (int c = 0; c < m; ++c) sum += al[c];
-    // 4. p = sum_c alpha_c x_c
+    // 4. p = sum_c alpha_c x_c, as (sum_c e_c x_c) / sum_c e_c: one division per dim
     double p[N];
 #pragma unroll
     for (int e = 0; e < N; ++e) p[e] = 0.0;
     for (int c = 0; c < m; ++c) {
-        const double a = al[c] / sum;
+        const double a = al[c];
         double x[N];
         load_dims<T, N>(sk + c * rs, off, x);
 #pragma unroll
         for (int e = 0; e < N; ++e) p[e] = fma(a, x[e], p[e]);
     }
+#pragma unroll
+    for (int e = 0; e < N; ++e) p[e] /= sum;
     // 5. the MLP input z = [mu / rho ; (p - mu) / sigma]; mu and p - mu kept for the end
 #pragma unroll
     for (int e = 0; e < N; ++e) {
