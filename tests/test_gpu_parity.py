@@ -406,3 +406,35 @@ def test_bounded_wait_gives_up_and_reports_timeout(R):
     assert int(st.item()) == 3
     run_decode_case(R, config_id=21, B=1, Hkv=1, Hq=2, d=64, C=4, k=3, lengths=[300],
                     dtype="f32", cap=300)
+
+
+def test_query_written_by_the_kernel_just_before_decode(R):
+    """The caller's own kernel may write q right before the decode on the same stream
+    (a projection or a RoPE kernel).  The decode is launched with programmatic
+    dependent launch and stages q only after its dependency wait, so it reads that
+    kernel's output: here q is written by a conversion kernel that follows a long
+    elementwise kernel, with no library kernel in between, and every output must equal
+    the one from a decode whose q was written and synchronised long before."""
+    C, k, d, Hkv, Hq, B, L0, steps = 16, 16, 128, 2, 8, 2, 6000, 4
+    cfg = R.Config(head_dim=d, n_q_heads=Hq, n_kv_heads=Hkv, C=C, k=k, dtype="bf16",
+                   pooler_w=H.w_for(C))
+    K, V, q_all = H.make_inputs(51, B, Hkv, Hq, d, L0, [L0] * B, "bf16", q_rows=steps)
+    tree = R.RecsaTree(cfg, L0, B, k0=K, v0=V)
+    tree.recsa_build([L0] * B)
+    ref = []
+    for s in range(steps):
+        qs = q_all[:, s].contiguous()
+        torch.cuda.synchronize()
+        ref.append(tree.decode(qs)[0].clone())
+    torch.cuda.synchronize()
+    big = torch.ones(64 << 20, dtype=torch.float32, device="cuda")   # 256 MB
+    src = [q_all[:, s].float().contiguous() for s in range(steps)]
+    qbuf = torch.empty_like(q_all[:, 0].contiguous())
+    torch.cuda.synchronize()
+    for s in range(steps):
+        big.mul_(1.0)        # a long kernel, so the next one ends late
+        qbuf.copy_(src[s])   # the kernel that writes q, launched right before the decode
+        out = tree.decode(qbuf)[0]
+        torch.cuda.synchronize()
+        assert tree.recsa_get_status() == R.RECSA_OK
+        assert torch.equal(out, ref[s]), f"step {s}: the decode read a stale query"
