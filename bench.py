@@ -100,6 +100,18 @@ def fp32_alu_peak():
     return 148 * 128 * 2 * mhz * 1e6 / 1e12, f"148 SMs x 128 fp32 lanes x 2 FLOP x {mhz:.0f} MHz"
 
 
+def fp64_alu_peak():
+    """Dense fp64 FMA rate of the CUDA cores, derived from unit counts and the clock:
+    148 SMs x 64 fp64 lanes x 2 FLOP per FMA x the measured max SM clock (MHz)."""
+    mhz = 1965.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    except Exception:
+        pass
+    return 148 * 64 * 2 * mhz * 1e6 / 1e12, f"148 SMs x 64 fp64 lanes x 2 FLOP x {mhz:.0f} MHz"
+
+
 def tf32_peak():
     """Dense tf32 tensor peak: the measured bf16 burst figure x the nominal tf32/bf16
     ratio (1.1 / 2.25 PFLOP/s), else the fallback 1.59 PFLOP/s x that ratio."""
@@ -650,8 +662,18 @@ def bench_gated_build(R, I, cfg, K, V, cap, B, L, dev, hidden=32):
     nodes = sum(B * W["Hkv"] * (-(-L // W["C"] ** l)) for l in range(1, 8) if -(-L // W["C"] ** (l - 1)) > 1)
     del tg
     torch.cuda.empty_cache()
+    # fp64 work per node with C children: the means (K and V: 2 C d adds), the
+    # projections and squared deviations (2 C d FMA), p (C d FMA), the MLP (2 d h + h d
+    # FMA), the output (2 d); counted as 2 FLOP per FMA and 1 per add
+    d, C = W["d"], W["C"]
+    flop_node = 2 * C * d + 2 * (2 * C * d + C * d + 3 * d * hidden) + 2 * d
+    peak, src = fp64_alu_peak()
+    achieved = flop_node * nodes / (ms / 1e3) / 1e12
     return {"ms": round(ms, 3), "hidden": hidden, "nodes": int(nodes),
             "ns_per_node": round(ms * 1e6 / nodes, 2),
+            "roofline": {"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_source": src, "flop_per_node": flop_node},
             "note": "Eq.5 gated key pooler, fp64, seeded parameters; values as Eq.1"}
 
 
