@@ -294,8 +294,9 @@ def run_ours(args):
     build_bytes = B * Hkv * L * d * esize * 2 * (1 + 1 / 15.0)
     gated = bench_gated_build(R, I, cfg, K, V, cap, B, L, dev)
 
-    # one decode step = append + decode, captured once; device-side lengths make
-    # the graph replayable step after step
+    # one decode step = recsa_append + recsa_decode, captured once; device-side lengths
+    # make the graph replayable step after step.  The same step as one call
+    # (recsa_append_decode, one launch) is timed beside it.
     kst = torch.empty(B, Hkv, 1, d, dtype=dt, device=dev)
     vst = torch.empty_like(kst)
     qst = torch.empty(B, Hq, d, dtype=dt, device=dev)
@@ -323,6 +324,10 @@ def run_ours(args):
                 tree.recsa_decode(qst, out, None, cnt)
         graphs[which] = gr
     tree.recsa_set_profile_events(0, None, None)
+    g_fused = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g_fused, stream=stream):
+            tree.recsa_append_decode(kst, vst, qst, out, None, cnt)
     torch.cuda.synchronize()
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -359,6 +364,21 @@ def run_ours(args):
         torch.cuda.synchronize()
         a, b_ = prof_ev[which]
         kern_ms[which].append(a.elapsed_time(b_))
+    # the same step as one call (append and pass in one launch), outside the timed
+    # region
+    fused_ms = []
+    for r in range(10):
+        qst.copy_(qs[r % S])
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        g_fused.replay()
+        s1.record()
+        s1.synchronize()
+        if r >= 2:
+            fused_ms.append(s0.elapsed_time(s1))
+    assert tree.recsa_get_status() == R.RECSA_OK
+    del g_fused
     ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
     value = whole_job_value(ms, ws, B)
     counts = cnt.cpu().numpy()
@@ -388,6 +408,9 @@ def run_ours(args):
                      "avg_launch_ms": round(kern_avg[dom], 5)},
         "kernel_ms": {("append" if w == -1 else "pass"):
                       (round(v, 5) if v else None) for w, v in kern_avg.items()},
+        "step": {"call": "recsa_append then recsa_decode (two launches)",
+                 "ms_one_call": round(sum(fused_ms) / len(fused_ms), 5),
+                 "one_call": "recsa_append_decode: the same step in one launch, same graph timing"},
         "build": {"ms": round(build_ms, 3), "GB_per_s": round(build_bytes / build_ms / 1e6, 1),
                   "tokens_per_seq": W["L"], "sequences": B},
         "build_gated": gated,

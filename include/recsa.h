@@ -158,6 +158,23 @@ RECSA_API recsa_status recsa_append(recsa_tree* tree, const void* k_new, const v
 RECSA_API recsa_status recsa_decode(recsa_tree* tree, const void* q, void* out, int32_t* sel_out,
                           int32_t* counts_out, void* stream);
 
+/* One decode step fused into one launch: the same as recsa_append(tree, k_new, v_new,
+ * 1, stream) followed by recsa_decode(tree, q, out, sel_out, counts_out, stream) --
+ * the same outputs, selections and counts, bit for bit, and the same tree afterwards
+ * ("Practical Implications": one token appended and attended per decode step).
+ *   k_new, v_new  device [B][Hkv][d] each, the token of every sequence (16-byte
+ *                 aligned); q, out, sel_out, counts_out as for recsa_decode.
+ * The walk CTAs of the launch write the token's rows at level 0 and re-pool its
+ * ancestors; the attention CTAs take the token's rows from k_new / v_new; the last CTA
+ * of each sequence advances its length.  Nothing is allocated; the caller keeps
+ * ownership of every buffer, which must stay valid until the stream reaches the call.
+ * Errors: RECSA_E_INVAL (null or misaligned pointer), RECSA_E_CAPACITY (a sequence
+ * at capacity), RECSA_E_UNSUPPORTED (a tree with the gated pooler or with level 0 in
+ * host memory: use the two separate calls), RECSA_E_CUDA (a launch failed). */
+RECSA_API recsa_status recsa_append_decode(recsa_tree* tree, const void* k_new, const void* v_new,
+                                           const void* q, void* out, int32_t* sel_out,
+                                           int32_t* counts_out, void* stream);
+
 /* Causal queries of a chunk: row i of sequence b sits at position pos0 + i and
  * must already be in the tree (pos0 + n <= L_b).
  *   Q  [batch][n][Hq][d] device;  O [batch][n][Hq][d] device.

@@ -467,6 +467,36 @@ recsa_status recsa_decode(recsa_tree* t, const void* q, void* out, int32_t* sel_
     return RECSA_OK;
 }
 
+recsa_status recsa_append_decode(recsa_tree* t, const void* k_new, const void* v_new,
+                                 const void* q, void* out, int32_t* sel_out, int32_t* counts_out,
+                                 void* stream) {
+    if (!t || !k_new || !v_new || !q || !out) return RECSA_E_INVAL;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q) || !aligned16(out))
+        return RECSA_E_INVAL;
+    // the separate calls serve the gated pooler and level 0 in host memory
+    if (t->gated || t->tv.l0_host) return RECSA_E_UNSUPPORTED;
+    for (int b = 0; b < t->B; ++b)
+        if (t->host_len[b] + 1 > t->cap) return RECSA_E_CAPACITY;
+    const cudaStream_t s = (cudaStream_t)stream;
+    if (finish_walk(t, s) != RECSA_OK) return RECSA_E_CUDA;   // an earlier append's walk
+    QueryView qv = {};
+    qv.q = q;
+    qv.out = out;
+    qv.sel_out = sel_out;
+    qv.cnt_out = counts_out;
+    qv.mode = 0;
+    qv.n_per_b = 1;
+    qv.nq = t->B;
+    qv.walk = 1;   // the walk CTAs write the token's rows and re-pool its ancestors
+    qv.knew = k_new;
+    qv.vnew = v_new;
+    cudaError_t e = launch_select_attend(t->tv, t->wv, qv, t->cfg.dtype, s, &t->prof,
+                                         t->has_maps ? t->maps : nullptr);
+    if (e != cudaSuccess) return RECSA_E_CUDA;
+    for (int b = 0; b < t->B; ++b) t->host_len[b] += 1;
+    return RECSA_OK;
+}
+
 // t / C^l and the first scored level of position t (host side of Eq.3's sizes).
 static int64_t host_apow(int64_t t, int l, int C) {
     for (int i = 0; i < l; ++i) t /= C;

@@ -88,6 +88,12 @@ struct QueryView {
     int phase;
     const void* l0k;
     const void* l0v;
+    // decode only, fused with a one-token append (non-null: [B][Hkv][D] each): the
+    // token goes to position t = the current length, the walk CTAs write its rows at
+    // level 0 and re-pool its ancestors, the attention CTAs take its rows from here,
+    // and the last CTA of each sequence advances the length
+    const void* knew;
+    const void* vnew;
 };
 
 // TMA tensor maps of one level's K and V tables (bf16, d = 128): 4-d (d, row, KV

@@ -1384,6 +1384,37 @@ struct PassMaps {
     KVMaps m[kMapLevels];
 };
 
+// Fused append: every CTA that reads lens[b] (the sequence's attention CTAs and its
+// walk CTAs, Hkv * (csize + 1) in all) counts itself once it has; the last one stores
+// the new length t + 1.  One thread per CTA, after a CTA barrier that follows the
+// reads.
+__device__ __forceinline__ void fused_count(const TreeView& tv, const WorkView& wv, int b,
+                                            int64_t t, int csize) {
+    __threadfence();
+    if (atomicAdd(&wv.done[b], 1u) == (unsigned)(tv.Hkv * (csize + 1)) - 1u) {
+        wv.done[b] = 0u;
+        wv.lens[b] = t + 1;
+    }
+}
+
+// Fused append: row r of a staged block (C rows, plain or swizzled) replaced by the
+// new token's row; lanes 0..D*esize/16-1 each store 16 bytes.  The stores are fenced
+// against the slot's next tensor copy.
+template <typename T, int D, bool SW>
+__device__ __forceinline__ void patch_row(unsigned char* blk, int r, int C, const T* row) {
+    constexpr int NCH = D * (int)sizeof(T) / 16;
+    const int lane = threadIdx.x & 31;
+    if (lane < NCH) {
+        const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(row) + 16 * lane);
+        uint32_t off;
+        if constexpr (SW) off = swz_off(lane >> 3, r, lane & 7, C);
+        else off = (uint32_t)(r * D * (int)sizeof(T) + 16 * lane);
+        *reinterpret_cast<uint4*>(blk + off) = v;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+}
+
 template <typename T, int D, int G, bool SW>
 __global__ void __launch_bounds__(kThreads, 2)
     pass_kernel(TreeView tv, WorkView wv, QueryView qv, const __grid_constant__ PassMaps maps,
@@ -1399,9 +1430,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         pdl_wait();
         for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
         const int b = ci / tv.Hkv, h = ci % tv.Hkv;
-        const int64_t t = wv.lens[b] - 1;
+        const bool fused = qv.knew != nullptr;
+        const int64_t t = fused ? wv.lens[b] : wv.lens[b] - 1;
+        if (fused && t < tv.cap) {
+            // the new token's rows at level 0, read back by this CTA's walk
+            constexpr int VEC = VecOf<T>::N;
+            const int64_t o = b * tv.s_b + h * tv.s_h + t * tv.s_t;
+            const T* kn = reinterpret_cast<const T*>(qv.knew) + ((int64_t)b * tv.Hkv + h) * D;
+            const T* vn = reinterpret_cast<const T*>(qv.vnew) + ((int64_t)b * tv.Hkv + h) * D;
+            for (int e = threadIdx.x; e < D / VEC; e += kThreads) {
+                *reinterpret_cast<uint4*>(reinterpret_cast<T*>(tv.k0w) + o + e * VEC) =
+                    *reinterpret_cast<const uint4*>(kn + e * VEC);
+                *reinterpret_cast<uint4*>(reinterpret_cast<T*>(tv.v0w) + o + e * VEC) =
+                    *reinterpret_cast<const uint4*>(vn + e * VEC);
+            }
+        }
         __syncthreads();
-        if (t >= 1) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha, wv.status);
+        if (fused && threadIdx.x == 0) fused_count(tv, wv, b, t, (int)gridDim.x);
+        if (t >= 1 && t < tv.cap) ancestor_walk<T, D, 4>(tv, b, h, t, pre, alpha, wv.status);
         return;
     }
     constexpr int kRow = D * (int)sizeof(T);
@@ -1493,8 +1539,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     pdl_wait();
     const int64_t len = wv.lens[b];
     stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
-    const int64_t t = (qv.mode == 0) ? len - 1 : qv.pos0 + (gq - b * qv.n_per_b);
-    const bool valid = t >= 0 && t < len;
+    const bool fused = qv.knew != nullptr;   // decode fused with a one-token append
+    const int64_t t = (qv.mode == 0) ? (fused ? len : len - 1) : qv.pos0 + (gq - b * qv.n_per_b);
+    const bool valid = t >= 0 && t < (fused ? tv.cap : len);
     const int lstar = valid ? first_scored_level(t, C, lgC, k) : 0;
     // the list geometry of every level, one thread per level (each a chain of
     // dependent integer steps): |A^(l)|, the entries per CTA, and the parents per
@@ -1516,6 +1563,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     float* part = wv.part + (int64_t)unit * wv.NSLOT * G * (D + 2);
     T* out = reinterpret_cast<T*>(qv.out) + ((int64_t)gq * tv.Hq + kvh * G) * D;
     __syncthreads();
+    if (fused && threadIdx.x == 0) fused_count(tv, wv, b, t, csize);
+    // fused append: the new token (entry |A^(0)|-1, the level-0 list's last) is staged
+    // from these rows instead of the cache, which its walk CTA is writing meanwhile
+    const T* knew_row = fused ? reinterpret_cast<const T*>(qv.knew) + ((int64_t)b * tv.Hkv + kvh) * D : nullptr;
+    const T* vnew_row = fused ? reinterpret_cast<const T*>(qv.vnew) + ((int64_t)b * tv.Hkv + kvh) * D : nullptr;
 
     if (!valid) {
         // nothing to attend (empty sequence, or a prefill row beyond the length):
@@ -1692,6 +1744,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const unsigned char* blk = ring_wait(R, qbase + i);
                 const int jb = j0 + (warp + kWarps * i) * C;
                 const int nch = min(C, j0 + n_sc - jb);
+                if (fused && L0 && jb <= nA - 1 && nA - 1 < jb + C)
+                    patch_row<T, D, SW>(const_cast<unsigned char*>(blk), nA - 1 - jb, C, knew_row);
                 float4 qn[CPL];
                 if (i + 1 < nw) load_qcs(jb + kWarps * C, qn);
                 if (nch > 0)
@@ -1771,6 +1825,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const unsigned char* blk = ring_wait(R, qbase + q);
                 const int jb = j0 + (warp + kWarps * i) * C;
                 const int nrow = min(C, j0 + n_sc - jb);
+                if (fused && L0 && jb <= nA - 1 && nA - 1 < jb + C)
+                    patch_row<T, D, SW>(const_cast<unsigned char*>(blk), nA - 1 - jb, C, vnew_row);
                 if (nrow > 0 && fm[0] > -INFINITY)
                     accum_parent_mma<D, G>(blk, C, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
                 __syncwarp();
@@ -1789,6 +1845,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const unsigned char* blk = ring_wait(R, qbase + q);
                 const int jb = j0 + (warp + kWarps * i) * C;
                 const int nrow = min(C, j0 + n_sc - jb);
+                if (fused && L0 && jb <= nA - 1 && nA - 1 < jb + C)
+                    patch_row<T, D, SW>(const_cast<unsigned char*>(blk), nA - 1 - jb, C, vnew_row);
                 if (nrow > 0 && fm[0] > -INFINITY)
                     accum_parent<T, D, G>(blk, jb, j0, nrow, L0 ? nullptr : flag, s, CH, acc);
                 __syncwarp();

@@ -81,6 +81,7 @@ def _load():
         "recsa_build": [P, ctypes.POINTER(I64), P],
         "recsa_append": [P, P, P, I32, P],
         "recsa_decode": [P, P, P, P, P, P],
+        "recsa_append_decode": [P, P, P, P, P, P, P, P],
         "recsa_prefill_chunk": [P, P, I64, I32, P, P, P, P],
         "recsa_get_status": [P, P],
         "recsa_tree_info": [P, ctypes.POINTER(RecsaTreeInfoC)],
@@ -236,6 +237,14 @@ class RecsaTree:
         assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.shape == v_new.shape
         _check(lib.recsa_append(self.handle, _ptr(k_new), _ptr(v_new), n, _stream(stream)),
                "recsa_append")
+
+    def recsa_append_decode(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                            out: torch.Tensor, sel_out=None, counts_out=None, stream=None):
+        assert k_new.is_contiguous() and v_new.is_contiguous() and k_new.shape == v_new.shape
+        assert k_new.shape[2] == 1 and q.is_contiguous() and out.is_contiguous()
+        _check(lib.recsa_append_decode(self.handle, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out),
+                                       _ptr(sel_out), _ptr(counts_out), _stream(stream)),
+               "recsa_append_decode")
 
     def recsa_decode(self, q: torch.Tensor, out: torch.Tensor, sel_out=None, counts_out=None,
                      stream=None):
