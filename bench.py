@@ -32,11 +32,11 @@ METRIC = "RecSA attn decode tok/s & prefill tok/s at 524K ctx; % HBM roofline"
 # capture at batch 1 (the pass kernel's summary under profiles/); a launch covers
 # batch x 8 independent units, so the batch-B figure is B times this.  Valid only
 # for the kernel sources it was taken from: any edit to them turns it into null.
-TRAFFIC_PASS_B1 = {"bytes": 44_191_744 + 81_152,
+TRAFFIC_PASS_B1 = {"bytes": 44_191_232 + 105_472,
                    "sources": ["long_context_recsa_b200/csrc/select_attend.cu",
                                "long_context_recsa_b200/csrc/recsa_internal.cuh",
                                "long_context_recsa_b200/csrc/pool.cuh"],
-                   "sha256": "0ea3d778045656719c8ea1623c1ea54fefccd865f4129100bbf26796669137d7"}
+                   "sha256": "885c99b5786e1e32301bd4041db2bf49f4c323f22f02c1988eaa4033d7c792aa"}
 
 
 def captured_traffic(kernel: str, batch: int):

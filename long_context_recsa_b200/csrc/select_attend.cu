@@ -1415,7 +1415,9 @@ __device__ __forceinline__ void patch_row(unsigned char* blk, int r, int C, cons
     __syncwarp();
 }
 
-template <typename T, int D, int G, bool SW>
+// FU: the decode fused with a one-token append (a separate instantiation, so that the
+// other launches carry none of its checks)
+template <typename T, int D, int G, bool SW, bool FU>
 __global__ void __launch_bounds__(kThreads, 2)
     pass_kernel(TreeView tv, WorkView wv, QueryView qv, const __grid_constant__ PassMaps maps,
                 int CH, int NA, int nsw) {
@@ -1430,7 +1432,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         pdl_wait();
         for (int i = threadIdx.x; i < tv.C * tv.C; i += kThreads) alpha[i] = wv.alpha[i];
         const int b = ci / tv.Hkv, h = ci % tv.Hkv;
-        const bool fused = qv.knew != nullptr;
+        const bool fused = FU && qv.knew != nullptr;
         const int64_t t = fused ? wv.lens[b] : wv.lens[b] - 1;
         if (fused && t < tv.cap) {
             // the new token's rows at level 0, read back by this CTA's walk
@@ -1539,7 +1541,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     pdl_wait();
     const int64_t len = wv.lens[b];
     stage_query<T, D, G>(qrow, wv.rope, C, qsm, rc4);
-    const bool fused = qv.knew != nullptr;   // decode fused with a one-token append
+    const bool fused = FU && qv.knew != nullptr;   // decode fused with a one-token append
     const int64_t t = (qv.mode == 0) ? (fused ? len : len - 1) : qv.pos0 + (gq - b * qv.n_per_b);
     const bool valid = t >= 0 && t < (fused ? tv.cap : len);
     const int lstar = valid ? first_scored_level(t, C, lgC, k) : 0;
@@ -1911,15 +1913,20 @@ static size_t pass_smem(int C, int k, int splits, int nslot, int n_levels, bool 
     return sm > ws ? sm : ws;
 }
 
-template <typename T, int D, int G, bool SW>
-static cudaError_t prepare_variant(size_t sm, int SPL) {
-    cudaError_t e = cudaFuncSetAttribute(pass_kernel<T, D, G, SW>,
+template <typename T, int D, int G, bool SW, bool FU>
+static cudaError_t prepare_one(size_t sm, int SPL) {
+    cudaError_t e = cudaFuncSetAttribute(pass_kernel<T, D, G, SW, FU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     if (SPL > 8)
-        e = cudaFuncSetAttribute(pass_kernel<T, D, G, SW>,
+        e = cudaFuncSetAttribute(pass_kernel<T, D, G, SW, FU>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
+}
+template <typename T, int D, int G, bool SW>
+static cudaError_t prepare_variant(size_t sm, int SPL) {
+    cudaError_t e = prepare_one<T, D, G, SW, false>(sm, SPL);
+    return e == cudaSuccess ? prepare_one<T, D, G, SW, true>(sm, SPL) : e;
 }
 
 template <typename T, int D, int G>
@@ -1962,7 +1969,9 @@ static cudaError_t select_attend_variant(const TreeView& tv, const WorkView& wv,
     prof_mark(prof, 0, true, s);
     NvtxRange nv(qv.phase == 1 ? "recsa pass (levels >= 1)" : qv.phase == 2 ? "recsa pass (level 0)"
                  : "recsa pass");
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pass_kernel<T, D, G, SW>, tv, wv, qv, pm, CH, NA, nsw);
+    cudaError_t e = qv.knew != nullptr
+                        ? cudaLaunchKernelEx(&cfg, pass_kernel<T, D, G, SW, true>, tv, wv, qv, pm, CH, NA, nsw)
+                        : cudaLaunchKernelEx(&cfg, pass_kernel<T, D, G, SW, false>, tv, wv, qv, pm, CH, NA, nsw);
     prof_mark(prof, 0, false, s);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
