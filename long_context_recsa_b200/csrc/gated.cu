@@ -27,8 +27,12 @@ inline size_t gated_smem(int D, int h, int warps) {
     const size_t per_warp = 4 * (size_t)D + h + RECSA_MAX_C;
     return sizeof(double) * (weights + warps * per_warp);
 }
-// Warps per CTA: 8 when their scratch fits beside the weights, else 4.
-inline int gated_warps(int D, int h) { return gated_smem(D, h, 8) <= 227 * 1024 ? 8 : 4; }
+// Warps per CTA: as many of 16, 8 or 4 as fit beside the weights (a node's chains
+// of dependent fp64 FMAs on shared-memory operands leave each warp mostly waiting,
+// so residency is what hides the latency).
+inline int gated_warps(int D, int h) {
+    return gated_smem(D, h, 16) <= 227 * 1024 ? 16 : gated_smem(D, h, 8) <= 227 * 1024 ? 8 : 4;
+}
 
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
@@ -176,7 +180,7 @@ __device__ void gated_pool_node(const T* sk, const T* sv, int64_t rs, int m, con
 // length L_old) or every node of [0, L) (add == 0).  A persistent grid: each CTA
 // stages the weights once and its warps take nodes in turn.
 template <typename T, int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(512, 1)
     gated_level_kernel(TreeView tv, WorkView wv, GatedView gv, int lvl, int64_t add) {
     extern __shared__ __align__(16) double gsm[];
     const int h = gv.h;
